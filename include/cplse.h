@@ -1,0 +1,168 @@
+/*
+ * cplse: the data-parallel hot path of decode-context-parallel (DCP) attention
+ * and of Ulysses sequence parallelism, for NVIDIA B200 (sm_100a).
+ *
+ *   pack     form LSE = softmax_max + log(softmax_sum) while writing the
+ *            head-partitioned send packet (payload in one region, fp32 LSE in
+ *            another); invalid statistics give LSE = -inf
+ *   a2a      the all-to-all's block permutation, W ranks emulated on one GPU
+ *   combine  stable log-sum-exp merge of the W partial outputs
+ *   fused    pack -> a2a -> combine in one pass; the packet never exists
+ *   Ulysses  sequence-scatter/head-gather layout transform and its inverse
+ *
+ * Sources, cited by page title and section:
+ *  [DCP] vLLM-Ascend pull request "[Performance][Attention] Fuse local SFA LSE
+ *        formation into DCP pack", sections "What this PR does / why we need
+ *        it?" (Before/After pipelines: native fp32 softmax_max/softmax_sum ->
+ *        max/sum-aware DCP pack -> HCCL All2All -> stable combine; invalid
+ *        statistics) and "How was this patch tested?" (bf16 and fp16,
+ *        scatter_dim 0 and 1, head dim 512, non-contiguous output/max/sum
+ *        strides, graph capture with changed-input replay).
+ *  [ULY] FastVideo compare view "[perf] Probe H3 chunked all-to-all with
+ *        direct output slices": all_to_all_4D(x, 2, 1) maps [B, S/W, H, D] to
+ *        [B, S, H/W, D] and all_to_all_4D(x, 1, 2) maps back; results must be
+ *        byte-identical to the NCCL all-to-all.
+ *
+ * Conventions for every entry point:
+ *  - Notation: W ranks, T tokens, H heads, Hc = H / W, D head dim. Layouts
+ *    are row-major, last index fastest. A "row" is the D elements of one
+ *    (rank, token, head). Payload elements are bf16 or fp16 (2 bytes).
+ *  - Pointers are DEVICE pointers on the current CUDA device (host pointers
+ *    are rejected with CP_ERR_ARG). The caller allocates and owns every
+ *    buffer; the library never allocates, frees or synchronises.
+ *  - `stream` is a cudaStream_t (NULL: the legacy default stream). Calls only
+ *    enqueue work on it and return; results are ready when the stream is.
+ *    No call performs a host<->device copy or a host synchronisation.
+ *  - Outputs must not overlap inputs (CP_ERR_ALIAS).
+ *  - All validation happens on the host before any launch. A failing call
+ *    enqueues nothing, returns a negative cp_status and records a message
+ *    for cp_last_error(). A call with zero rows (T == 0 or B == 0) is a
+ *    valid no-op. The library never aborts the process and has no device
+ *    side traps, asserts or waits.
+ */
+#ifndef CPLSE_H
+#define CPLSE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define CPLSE_API __attribute__((visibility("default")))
+#else
+#define CPLSE_API
+#endif
+
+#define CPLSE_ABI_VERSION 1
+#define CPLSE_MAX_W 32     /* simulated ranks per call */
+#define CPLSE_MAX_D 1024   /* head dim, elements */
+
+typedef enum cp_status {
+    CP_OK = 0,
+    CP_ERR_ARG = -1,          /* null/host pointer, bad enum, negative size */
+    CP_ERR_SHAPE = -2,        /* H % W, T % W, S_local, D % 8 ... */
+    CP_ERR_ALIGN = -3,        /* base not 16-byte aligned, stride not a multiple of 8 elements */
+    CP_ERR_ALIAS = -4,        /* an output overlaps an input */
+    CP_ERR_UNSUPPORTED = -5,  /* W > 32, D > 1024, ... */
+    CP_ERR_CUDA = -6          /* the launch itself failed (message has the CUDA error) */
+} cp_status;
+
+typedef enum cp_dtype { CP_BF16 = 0, CP_FP16 = 1 } cp_dtype;
+
+/* Element strides of a [W][T][H] (or [W][T][H][D] with D contiguous) view. */
+typedef struct cp_strides3 {
+    int64_t r, t, h;
+} cp_strides3;
+
+/* CPLSE_ABI_VERSION of the loaded library. */
+CPLSE_API int cp_abi_version(void);
+
+/* Message of the last failing call on this host thread ("" if none). The
+ * pointer stays valid until the next call on the same thread. */
+CPLSE_API const char* cp_last_error(void);
+
+/*
+ * [DCP] "max/sum-aware DCP pack, which forms the same LSE while writing the
+ * packed layout" (After pipeline), with the invalid-statistic rule of the same
+ * section: a non-finite softmax_max, a non-finite softmax_sum or a
+ * softmax_sum <= 0 gives LSE = -inf. LSE = max + logf(sum) in fp32.
+ *
+ *   o      payload [W][T][H][D], element strides `so` (D contiguous; so.* >= 0
+ *          and multiples of 8; base 16-byte aligned)
+ *   smax   fp32 [W][T][H], element strides `sm` (>= 0, any value)
+ *   ssum   fp32 [W][T][H], element strides `ss`
+ *   scatter_dim 1 (head chunks, the DCP path; H % W == 0):
+ *            pkt_o   [W_src][W_dst][T][Hc][D]   pkt_o[r][j][t][hc] = o[r][t][j*Hc+hc]
+ *            pkt_lse [W_src][W_dst][T][Hc]      fp32
+ *   scatter_dim 0 (token chunks; T % W == 0, Tc = T / W):
+ *            pkt_o   [W_src][W_dst][Tc][H][D]   pkt_o[r][j][tc][h] = o[r][j*Tc+tc][h]
+ *            pkt_lse [W_src][W_dst][Tc][H]
+ *   Payload bits are copied unchanged. pkt_o: 16-byte aligned, contiguous.
+ */
+CPLSE_API cp_status cp_pack_lse(const void* o, cp_strides3 so, const float* smax, cp_strides3 sm,
+                      const float* ssum, cp_strides3 ss, int W, int64_t T, int H, int D,
+                      cp_dtype dt, int scatter_dim, void* pkt_o, float* pkt_lse, void* stream);
+
+/*
+ * [DCP] "HCCL All2All" of the packet, emulated on one GPU: W simulated ranks
+ * each hold W blocks of `block_bytes`; block j of rank r lands as block r of
+ * rank j:  recv[j][r] = send[r][j]. Call it once per packet region (payload
+ * block = T*Hc*D*2 bytes, LSE block = T*Hc*4 bytes). Any block size works;
+ * 16-byte aligned bases with block_bytes % 16 == 0 take the vector path.
+ */
+CPLSE_API cp_status cp_a2a_local_permute(const void* send, void* recv, int W, int64_t block_bytes,
+                               void* stream);
+
+/*
+ * [DCP] the stable combine each destination rank runs on what it received.
+ *   recv_o   [W_dst][W_src][N][D] payload, N = T*Hc rows per block
+ *   recv_lse [W_dst][W_src][N]    fp32, each finite or -inf (NaN counts as -inf)
+ *   out      [W_dst][N][D]        payload dtype, fp32 accumulation, nearest-even
+ *   out_lse  [W_dst][N]           fp32
+ * Per output row, over r = 0..W-1: M = max lse_r; if M = -inf the row is all
+ * invalid: out = +0, out_lse = -inf. Otherwise LSE* = M + logf(sum_r expf(lse_r - M)),
+ * out = sum_r expf(lse_r - LSE*) * o_r over the valid r only (an invalid
+ * contribution's payload is never read into the sum). For the token-chunk
+ * packet pass T/W as T and H as Hc.
+ */
+CPLSE_API cp_status cp_lse_combine(const void* recv_o, const float* recv_lse, int W, int64_t T, int Hc,
+                         int D, cp_dtype dt, void* out, float* out_lse, void* stream);
+
+/*
+ * pack (head chunks) -> a2a -> combine in one pass: output row (j, t, hc)
+ * reads row (t, j*Hc + hc) of every rank's o/smax/ssum directly. Inputs as in
+ * cp_pack_lse; outputs as in cp_lse_combine with N = T*Hc:
+ *   out [W][T][Hc][D], out_lse [W][T][Hc].
+ * Bit-identical to cp_pack_lse(scatter_dim=1) -> cp_a2a_local_permute (both
+ * regions) -> cp_lse_combine.
+ */
+CPLSE_API cp_status cp_pack_permute_combine_fused(const void* o, cp_strides3 so, const float* smax,
+                                        cp_strides3 sm, const float* ssum, cp_strides3 ss, int W,
+                                        int64_t T, int H, int D, cp_dtype dt, void* out,
+                                        float* out_lse, void* stream);
+
+/*
+ * [ULY] all_to_all_4D(x, scatter_dim=2, gather_dim=1), W ranks on one GPU:
+ *   in  [W][B][S_local][H][D]  ->  out [W][B][W*S_local][H/W][D]
+ *   out[j][b][r*S_local + s][hc] = in[r][b][s][j*Hc + hc]
+ * A byte copy of elem_bytes-sized elements (1, 2, 4 or 8); H % W == 0.
+ */
+CPLSE_API cp_status ulysses_seq2head(const void* in, void* out, int W, int B, int64_t S_local, int H, int D,
+                           int elem_bytes, void* stream);
+
+/*
+ * [ULY] all_to_all_4D(x, scatter_dim=1, gather_dim=2), the inverse:
+ *   in  [W][B][W*S_local][H/W][D]  ->  out [W][B][S_local][H][D]
+ *   out[j][b][s][r*Hc + hc] = in[r][b][j*S_local + s][hc]
+ * ulysses_head2seq(ulysses_seq2head(x)) == x.
+ */
+CPLSE_API cp_status ulysses_head2seq(const void* in, void* out, int W, int B, int64_t S_local, int H, int D,
+                           int elem_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CPLSE_H */

@@ -1,0 +1,206 @@
+"""Python binding of libcplse (include/cplse.h): argument marshalling only.
+
+Every function has the name of its C entry point, takes torch CUDA tensors,
+passes their device pointers, sizes and strides through the C-ABI, and
+enqueues the work on the current torch stream (or ``stream=``). Outputs are
+allocated with ``torch.empty`` when not given. Nothing here computes any part
+of the method: there is no fallback path. If the shared library is missing or
+a call fails, a ``RuntimeError`` carries the library's message.
+
+Layouts (W ranks, T tokens, H heads, Hc = H/W, D head dim):
+    o            [W, T, H, D]   bf16/fp16, D contiguous, other strides free
+    smax, ssum   [W, T, H]      float32, any strides
+    pkt_o        [W, W, T, Hc, D] (heads) or [W, W, T/W, H, D] (tokens)
+    pkt_lse      [W, W, T, Hc]    or [W, W, T/W, H]   float32
+    out          [W, T, Hc, D],  out_lse [W, T, Hc]
+    Ulysses      [W, B, S/W, H, D] <-> [W, B, S, Hc, D]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_HERE, "libcplse.so")
+
+if not os.path.exists(LIBRARY_PATH):
+    raise ImportError("libcplse.so is not built: run `python -m lse_pack_stable_b200.build` "
+                      "(or __graft_entry__.build())")
+
+_lib = ctypes.CDLL(LIBRARY_PATH)
+
+CP_OK, CP_ERR_ARG, CP_ERR_SHAPE, CP_ERR_ALIGN, CP_ERR_ALIAS, CP_ERR_UNSUPPORTED, CP_ERR_CUDA = (
+    0, -1, -2, -3, -4, -5, -6)
+CP_BF16, CP_FP16 = 0, 1
+STATUS_NAMES = {0: "CP_OK", -1: "CP_ERR_ARG", -2: "CP_ERR_SHAPE", -3: "CP_ERR_ALIGN",
+                -4: "CP_ERR_ALIAS", -5: "CP_ERR_UNSUPPORTED", -6: "CP_ERR_CUDA"}
+EXPORTS = ("cp_abi_version", "cp_last_error", "cp_pack_lse", "cp_a2a_local_permute",
+           "cp_lse_combine", "cp_pack_permute_combine_fused", "ulysses_seq2head",
+           "ulysses_head2seq")
+
+
+class Strides3(ctypes.Structure):
+    _fields_ = [("r", ctypes.c_int64), ("t", ctypes.c_int64), ("h", ctypes.c_int64)]
+
+
+_p, _i, _i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+_lib.cp_abi_version.argtypes = []
+_lib.cp_abi_version.restype = _i
+_lib.cp_last_error.argtypes = []
+_lib.cp_last_error.restype = ctypes.c_char_p
+_lib.cp_pack_lse.argtypes = [_p, Strides3, _p, Strides3, _p, Strides3, _i, _i64, _i, _i, _i, _i,
+                             _p, _p, _p]
+_lib.cp_a2a_local_permute.argtypes = [_p, _p, _i, _i64, _p]
+_lib.cp_lse_combine.argtypes = [_p, _p, _i, _i64, _i, _i, _i, _p, _p, _p]
+_lib.cp_pack_permute_combine_fused.argtypes = [_p, Strides3, _p, Strides3, _p, Strides3, _i, _i64,
+                                               _i, _i, _i, _p, _p, _p]
+_lib.ulysses_seq2head.argtypes = [_p, _p, _i, _i, _i64, _i, _i, _i, _p]
+_lib.ulysses_head2seq.argtypes = [_p, _p, _i, _i, _i64, _i, _i, _i, _p]
+for _f in ("cp_pack_lse", "cp_a2a_local_permute", "cp_lse_combine",
+           "cp_pack_permute_combine_fused", "ulysses_seq2head", "ulysses_head2seq"):
+    getattr(_lib, _f).restype = _i
+
+
+class CplseError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__("%s: %s" % (STATUS_NAMES.get(status, status), message))
+        self.status = status
+
+
+def _check(status: int) -> None:
+    if status != CP_OK:
+        raise CplseError(status, _lib.cp_last_error().decode())
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return CP_BF16
+    if t.dtype == torch.float16:
+        return CP_FP16
+    raise TypeError("payload dtype must be bfloat16 or float16, got %s" % t.dtype)
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _strides3(t: torch.Tensor) -> Strides3:
+    st = t.stride()
+    if t.dim() == 4 and st[3] != 1:
+        raise ValueError("the head dim (last) of o must be contiguous")
+    return Strides3(st[0], st[1], st[2])
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _dense(t: torch.Tensor, name: str) -> None:
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def abi_version() -> int:
+    return _lib.cp_abi_version()
+
+
+def last_error() -> str:
+    return _lib.cp_last_error().decode()
+
+
+def cp_pack_lse(o: torch.Tensor, smax: torch.Tensor, ssum: torch.Tensor, scatter_dim: int = 1,
+                pkt_o: Optional[torch.Tensor] = None, pkt_lse: Optional[torch.Tensor] = None,
+                stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    W, T, H, D = o.shape
+    if scatter_dim == 1:
+        shape = (W, W, T, H // W)
+    else:
+        shape = (W, W, T // W, H)
+    if pkt_o is None:
+        pkt_o = torch.empty(shape + (D,), dtype=o.dtype, device=o.device)
+    if pkt_lse is None:
+        pkt_lse = torch.empty(shape, dtype=torch.float32, device=o.device)
+    _dense(pkt_o, "pkt_o")
+    _dense(pkt_lse, "pkt_lse")
+    _check(_lib.cp_pack_lse(_ptr(o), _strides3(o), _ptr(smax), _strides3(smax), _ptr(ssum),
+                            _strides3(ssum), W, T, H, D, _dtype(o), scatter_dim, _ptr(pkt_o),
+                            _ptr(pkt_lse), _stream(stream)))
+    return pkt_o, pkt_lse
+
+
+def cp_a2a_local_permute(send: torch.Tensor, W: int, recv: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """send: any contiguous tensor whose bytes are W*W equal blocks [src][dst]."""
+    if recv is None:
+        recv = torch.empty_like(send)
+    _dense(send, "send")
+    _dense(recv, "recv")
+    nbytes = send.numel() * send.element_size()
+    if nbytes % (W * W) != 0:
+        raise ValueError("send bytes (%d) are not W*W equal blocks" % nbytes)
+    _check(_lib.cp_a2a_local_permute(_ptr(send), _ptr(recv), W, nbytes // (W * W),
+                                     _stream(stream)))
+    return recv
+
+
+def cp_lse_combine(recv_o: torch.Tensor, recv_lse: torch.Tensor,
+                   out: Optional[torch.Tensor] = None, out_lse: Optional[torch.Tensor] = None,
+                   stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """recv_o [W, W, T, Hc, D], recv_lse [W, W, T, Hc] -> out [W, T, Hc, D], out_lse [W, T, Hc]."""
+    W, W2, T, Hc, D = recv_o.shape
+    if out is None:
+        out = torch.empty((W, T, Hc, D), dtype=recv_o.dtype, device=recv_o.device)
+    if out_lse is None:
+        out_lse = torch.empty((W, T, Hc), dtype=torch.float32, device=recv_o.device)
+    for t, n in ((recv_o, "recv_o"), (recv_lse, "recv_lse"), (out, "out"), (out_lse, "out_lse")):
+        _dense(t, n)
+    _check(_lib.cp_lse_combine(_ptr(recv_o), _ptr(recv_lse), W, T, Hc, D, _dtype(recv_o),
+                               _ptr(out), _ptr(out_lse), _stream(stream)))
+    return out, out_lse
+
+
+def cp_pack_permute_combine_fused(o: torch.Tensor, smax: torch.Tensor, ssum: torch.Tensor,
+                                  out: Optional[torch.Tensor] = None,
+                                  out_lse: Optional[torch.Tensor] = None,
+                                  stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    W, T, H, D = o.shape
+    if out is None:
+        out = torch.empty((W, T, H // W, D), dtype=o.dtype, device=o.device)
+    if out_lse is None:
+        out_lse = torch.empty((W, T, H // W), dtype=torch.float32, device=o.device)
+    _dense(out, "out")
+    _dense(out_lse, "out_lse")
+    _check(_lib.cp_pack_permute_combine_fused(_ptr(o), _strides3(o), _ptr(smax), _strides3(smax),
+                                              _ptr(ssum), _strides3(ssum), W, T, H, D, _dtype(o),
+                                              _ptr(out), _ptr(out_lse), _stream(stream)))
+    return out, out_lse
+
+
+def ulysses_seq2head(x: torch.Tensor, out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """x [W, B, S/W, H, D] (contiguous) -> [W, B, S, H/W, D]."""
+    W, B, S_l, H, D = x.shape
+    if out is None:
+        out = torch.empty((W, B, S_l * W, H // W, D), dtype=x.dtype, device=x.device)
+    _dense(x, "x")
+    _dense(out, "out")
+    _check(_lib.ulysses_seq2head(_ptr(x), _ptr(out), W, B, S_l, H, D, x.element_size(),
+                                 _stream(stream)))
+    return out
+
+
+def ulysses_head2seq(x: torch.Tensor, out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """x [W, B, S, Hc, D] (contiguous) -> [W, B, S/W, Hc*W, D]."""
+    W, B, S, Hc, D = x.shape
+    if out is None:
+        out = torch.empty((W, B, S // W, Hc * W, D), dtype=x.dtype, device=x.device)
+    _dense(x, "x")
+    _dense(out, "out")
+    _check(_lib.ulysses_head2seq(_ptr(x), _ptr(out), W, B, S // W, Hc * W, D, x.element_size(),
+                                 _stream(stream)))
+    return out

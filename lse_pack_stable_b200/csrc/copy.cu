@@ -1,0 +1,180 @@
+// Layout kernels that move bytes without arithmetic:
+//  - the all-to-all's block permutation between W simulated ranks
+//    (vLLM-Ascend "Fuse local SFA LSE formation into DCP pack", Before/After
+//    pipelines: the HCCL All2All of the packed layout);
+//  - the Ulysses sequence-scatter/head-gather transform and its inverse
+//    (FastVideo "[perf] Probe H3 chunked all-to-all with direct output
+//    slices": all_to_all_4D(x, 2, 1) and all_to_all_4D(x, 1, 2)).
+// Every access is the widest vector (16, 8, 4, 2 or 1 bytes) that the block
+// size and both base addresses allow; several loads are in flight per thread
+// before the first store.
+#include "common.cuh"
+#include "launch.h"
+
+namespace cplse {
+namespace {
+
+constexpr int kCopyThreads = 256;
+
+template <typename V>
+__device__ __forceinline__ V ld_cs(const V* p) { return __ldcs(p); }
+template <typename V>
+__device__ __forceinline__ void st_cs(V* p, V v) { __stcs(p, v); }
+
+// recv[j][r] = send[r][j]; grid.y enumerates destination blocks d = j*W + r.
+template <typename V, int U>
+__global__ void __launch_bounds__(kCopyThreads)
+permute_kernel(const V* __restrict__ send, V* __restrict__ recv, int W, int64_t nvec)
+{
+    const int d = blockIdx.y;
+    const int j = d / W, r = d - j * W;
+    const V* src = send + (int64_t)(r * W + j) * nvec;
+    V* dst = recv + (int64_t)d * nvec;
+    const int64_t stride = (int64_t)gridDim.x * kCopyThreads * U;
+    for (int64_t base = (int64_t)blockIdx.x * kCopyThreads * U + threadIdx.x; base < nvec;
+         base += stride) {
+        V v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + (int64_t)u * kCopyThreads;
+            if (i < nvec) v[u] = ld_cs(src + i);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + (int64_t)u * kCopyThreads;
+            if (i < nvec) st_cs(dst + i, v[u]);
+        }
+    }
+}
+
+template <typename V>
+cudaError_t launch_permute_v(const void* send, void* recv, int W, int64_t block_bytes,
+                             cudaStream_t s)
+{
+    constexpr int U = 4;
+    const int64_t nvec = block_bytes / (int64_t)sizeof(V);
+    int64_t gx = (nvec + kCopyThreads * U - 1) / (kCopyThreads * U);
+    // enough CTAs to fill every SM several times over; the rest is grid-stride
+    const int64_t want = (int64_t)sm_count() * 16;
+    const int64_t per_block_cap = (want + (int64_t)W * W - 1) / ((int64_t)W * W);
+    if (gx > per_block_cap) gx = per_block_cap;
+    if (gx < 1) gx = 1;
+    dim3 grid((unsigned)gx, (unsigned)(W * W));
+    permute_kernel<V, U><<<grid, kCopyThreads, 0, s>>>(static_cast<const V*>(send),
+                                                      static_cast<V*>(recv), W, nvec);
+    return cudaGetLastError();
+}
+
+// One warp per contiguous chunk of Hc*D elements.
+//   mode 0 (seq->head): chunk c = ((r*B + b)*S_l + s)*W + j of the input
+//       lands at chunk (j*B + b)*S + r*S_l + s of the output;
+//   mode 1 (head->seq): chunk c = (r*B + b)*S + (j*S_l + s) of the input
+//       lands at chunk ((j*B + b)*S_l + s)*W + r of the output.
+template <typename V, int MODE, int UNR>
+__global__ void __launch_bounds__(kCopyThreads)
+ulysses_kernel(const V* __restrict__ in, V* __restrict__ out, const UlyssesArgs a, int64_t cv)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = ((int64_t)blockIdx.x * kCopyThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * kCopyThreads) >> 5;
+    for (int64_t c = warp; c < a.nchunks; c += nwarps) {
+        int64_t dc;
+        if (MODE == 0) {
+            int64_t rest = c / a.W;
+            const int64_t j = c - rest * a.W;
+            const int64_t s = rest % a.S_l;
+            rest /= a.S_l;
+            const int64_t b = rest % a.B;
+            const int64_t r = rest / a.B;
+            dc = (j * a.B + b) * a.S + r * a.S_l + s;
+        } else {
+            int64_t rest = c / a.S;
+            const int64_t sg = c - rest * a.S;
+            const int64_t b = rest % a.B;
+            const int64_t r = rest / a.B;
+            const int64_t j = sg / a.S_l;
+            const int64_t s = sg - j * a.S_l;
+            dc = ((j * a.B + b) * a.S_l + s) * a.W + r;
+        }
+        const V* src = in + c * cv;
+        V* dst = out + dc * cv;
+        for (int64_t v0 = lane; v0 < cv; v0 += 32 * UNR) {
+            V x[UNR];
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int64_t i = v0 + 32 * u;
+                if (i < cv) x[u] = ld_cs(src + i);
+            }
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int64_t i = v0 + 32 * u;
+                if (i < cv) st_cs(dst + i, x[u]);
+            }
+        }
+    }
+}
+
+template <typename V, int MODE>
+cudaError_t launch_ulysses_v(const UlyssesArgs& a, cudaStream_t s)
+{
+    constexpr int UNR = 4;
+    auto kern = ulysses_kernel<V, MODE, UNR>;
+    static int per_sm = 0;
+    if (per_sm == 0) {
+        int n = 0;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kCopyThreads, 0);
+        if (e != cudaSuccess) return e;
+        per_sm = n > 0 ? n : 1;
+    }
+    const int64_t cv = a.chunk_bytes / (int64_t)sizeof(V);
+    const int64_t warps_per_block = kCopyThreads / 32;
+    int64_t blocks = (a.nchunks + warps_per_block - 1) / warps_per_block;
+    const int64_t cap = (int64_t)per_sm * sm_count();
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    kern<<<(unsigned)blocks, kCopyThreads, 0, s>>>(static_cast<const V*>(a.in),
+                                                  static_cast<V*>(a.out), a, cv);
+    return cudaGetLastError();
+}
+
+// Widest power-of-two access (<= 16 bytes) dividing n and both addresses.
+int vector_bytes(int64_t n, const void* p, const void* q)
+{
+    const uint64_t m = (uint64_t)n | (uint64_t)(uintptr_t)p | (uint64_t)(uintptr_t)q;
+    for (int w = 16; w > 1; w >>= 1)
+        if ((m & (uint64_t)(w - 1)) == 0) return w;
+    return 1;
+}
+
+template <int MODE>
+cudaError_t launch_ulysses_m(const UlyssesArgs& a, cudaStream_t s)
+{
+    switch (vector_bytes(a.chunk_bytes, a.in, a.out)) {
+    case 16: return launch_ulysses_v<uint4, MODE>(a, s);
+    case 8: return launch_ulysses_v<uint2, MODE>(a, s);
+    case 4: return launch_ulysses_v<unsigned int, MODE>(a, s);
+    case 2: return launch_ulysses_v<unsigned short, MODE>(a, s);
+    default: return launch_ulysses_v<unsigned char, MODE>(a, s);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const void* send, void* recv, int W, int64_t block_bytes,
+                           cudaStream_t s)
+{
+    switch (vector_bytes(block_bytes, send, recv)) {
+    case 16: return launch_permute_v<uint4>(send, recv, W, block_bytes, s);
+    case 8: return launch_permute_v<uint2>(send, recv, W, block_bytes, s);
+    case 4: return launch_permute_v<unsigned int>(send, recv, W, block_bytes, s);
+    case 2: return launch_permute_v<unsigned short>(send, recv, W, block_bytes, s);
+    default: return launch_permute_v<unsigned char>(send, recv, W, block_bytes, s);
+    }
+}
+
+cudaError_t launch_ulysses(const UlyssesArgs& a, cudaStream_t s)
+{
+    return a.mode == 0 ? launch_ulysses_m<0>(a, s) : launch_ulysses_m<1>(a, s);
+}
+
+}  // namespace cplse

@@ -1,0 +1,67 @@
+// Internal launcher interface between the C-ABI layer (api.cu) and the kernels.
+// Arguments arrive here already validated; launchers only pick a kernel
+// instantiation and a grid, enqueue, and report cudaGetLastError().
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace cplse {
+
+enum class Dtype : int { kBf16 = 0, kFp16 = 1 };
+
+// Stable log-sum-exp merge of W contributions per output row. FUSED mode forms
+// each contribution's LSE from (max, sum) and reads the partial outputs in
+// place; COMBINE mode reads a received packet.
+struct CombineArgs {
+    const uint16_t* src;      // payload base
+    int64_t rank_stride;      // elements between ranks' rows
+    // fused: o[r][t][h] at src + r*rank_stride + t*so_t + h*so_h
+    int64_t so_t, so_h;
+    const float* smax;
+    const float* ssum;
+    int64_t sm_r, sm_t, sm_h, ss_r, ss_t, ss_h;
+    // combine: recv_lse[j][r][n]
+    const float* lse;
+    uint16_t* out;
+    float* out_lse;
+    int W, H, Hc, D;
+    int64_t T;                // fused: tokens
+    int64_t N;                // combine: rows per block
+    int64_t rows;             // output rows
+};
+
+struct PackArgs {
+    const uint16_t* o;
+    int64_t so_r, so_t, so_h;
+    const float* smax;
+    const float* ssum;
+    int64_t sm_r, sm_t, sm_h, ss_r, ss_t, ss_h;
+    uint16_t* pkt_o;
+    float* pkt_lse;
+    int W, H, Hc, D, scatter_dim;
+    int64_t T, Tc;
+    int64_t rows;             // W*T*H
+};
+
+struct UlyssesArgs {
+    const void* in;
+    void* out;
+    int W, B, H, Hc;
+    int64_t S_l, S;
+    int64_t chunk_bytes;      // Hc*D*elem_bytes
+    int64_t nchunks;
+    int mode;                 // 0: seq->head, 1: head->seq
+};
+
+cudaError_t launch_fused(const CombineArgs& a, Dtype dt, cudaStream_t s);
+cudaError_t launch_combine(const CombineArgs& a, Dtype dt, cudaStream_t s);
+cudaError_t launch_pack(const PackArgs& a, cudaStream_t s);
+cudaError_t launch_permute(const void* send, void* recv, int W, int64_t block_bytes,
+                           cudaStream_t s);
+cudaError_t launch_ulysses(const UlyssesArgs& a, cudaStream_t s);
+
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count();
+
+}  // namespace cplse

@@ -1,0 +1,136 @@
+// Max/sum-aware DCP pack: forms LSE = softmax_max + log(softmax_sum) (-inf for
+// invalid statistics) while writing the destination-major send packet.
+//
+// Source: vLLM-Ascend pull request "[Performance][Attention] Fuse local SFA LSE
+// formation into DCP pack", section "What this PR does / why we need it?"
+// (After pipeline: the pack forms the same LSE while writing the packed layout;
+// invalid-statistic rule) and "How was this patch tested?" (scatter_dim 0 and
+// 1, non-contiguous output/max/sum strides).
+//
+// Work split: a warp owns chunks of 32 consecutive source rows (r, t, h) in
+// input order. Phase A: lane i forms the LSE of row i (coalesced max/sum
+// loads) and writes it to the LSE region. Phase B: G lanes copy one row's D
+// elements with 16-byte vectors; U steps of loads are in flight before the
+// first store.
+#include <math.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "rowcombine.cuh"
+
+namespace cplse {
+namespace {
+
+constexpr int kPackThreads = 128;
+
+template <int G, int VPL, int U>
+__global__ void __launch_bounds__(kPackThreads) pack_kernel(const PackArgs a)
+{
+    constexpr int RPI = 32 / G;
+    constexpr int STEPS = 32 / RPI;
+    static_assert(STEPS % U == 0, "U must divide the steps of a chunk");
+    const int lane = threadIdx.x & 31;
+    const int sub = lane / G;
+    const int gl = lane % G;
+    const int64_t warp = ((int64_t)blockIdx.x * kPackThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * kPackThreads) >> 5;
+    const int64_t nchunks = (a.rows + 31) >> 5;
+    const int V = a.D >> 3;
+    const int64_t TH = a.T * a.H;
+    const int64_t block_rows = a.T * a.Hc;   // rows of one [src][dst] packet block
+
+    for (int64_t c = warp; c < nchunks; c += nwarps) {
+        // ---------------- phase A: lane owns source row q = (r, t, h)
+        const int64_t q = c * 32 + lane;
+        const bool qv = q < a.rows;
+        int64_t src_row = 0, dst_row = 0;
+        if (qv) {
+            const int64_t r = q / TH;
+            const int64_t rem = q - r * TH;
+            const int64_t t = rem / a.H;
+            const int64_t h = rem - t * a.H;
+            int64_t j, slot;
+            if (a.scatter_dim == 1) {
+                j = h / a.Hc;
+                slot = t * a.Hc + (h - j * a.Hc);
+            } else {
+                j = t / a.Tc;
+                slot = (t - j * a.Tc) * a.H + h;
+            }
+            dst_row = (r * a.W + j) * block_rows + slot;
+            src_row = r * a.so_r + t * a.so_t + h * a.so_h;
+            const float m = ld_stream(a.smax + r * a.sm_r + t * a.sm_t + h * a.sm_h);
+            const float s = ld_stream(a.ssum + r * a.ss_r + t * a.ss_t + h * a.ss_h);
+            const bool ok = isfinite(m) && isfinite(s) && s > 0.f;
+            st_stream(a.pkt_lse + dst_row, ok ? m + logf(s) : -INFINITY);
+        }
+
+        // ---------------- phase B: copy the payload rows
+#pragma unroll 1
+        for (int s0 = 0; s0 < STEPS; s0 += U) {
+            int64_t sb[U], db[U];
+            bool rv[U];
+            uint4 v[U][VPL];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int k = (s0 + u) * RPI + sub;
+                sb[u] = __shfl_sync(kFull, src_row, k);
+                db[u] = __shfl_sync(kFull, dst_row, k);
+                rv[u] = c * 32 + k < a.rows;
+#pragma unroll
+                for (int e = 0; e < VPL; ++e) {
+                    const int vec = gl + e * G;
+                    if (rv[u] && vec < V)
+                        v[u][e] = ld_stream(reinterpret_cast<const uint4*>(a.o + sb[u]) + vec);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int e = 0; e < VPL; ++e) {
+                    const int vec = gl + e * G;
+                    if (rv[u] && vec < V)
+                        st_stream(reinterpret_cast<uint4*>(a.pkt_o + db[u] * a.D) + vec, v[u][e]);
+                }
+        }
+    }
+}
+
+template <int G, int VPL>
+cudaError_t launch_pack_inst(const PackArgs& a, cudaStream_t s)
+{
+    constexpr int U0 = VPL >= 8 ? 1 : 8 / VPL;
+    constexpr int U = U0 > G ? G : U0;
+    auto kern = pack_kernel<G, VPL, U>;
+    static int per_sm = 0;
+    if (per_sm == 0) {
+        int n = 0;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kPackThreads, 0);
+        if (e != cudaSuccess) return e;
+        per_sm = n > 0 ? n : 1;
+    }
+    const int64_t nchunks = (a.rows + 31) / 32;
+    int64_t blocks = (nchunks + kPackThreads / 32 - 1) / (kPackThreads / 32);
+    const int64_t cap = (int64_t)per_sm * sm_count();
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    kern<<<(unsigned)blocks, kPackThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const PackArgs& a, cudaStream_t s)
+{
+    const RowShape rs = row_shape(a.D);
+    switch (rs.G * 10 + rs.VPL) {
+    case 41: return launch_pack_inst<4, 1>(a, s);
+    case 81: return launch_pack_inst<8, 1>(a, s);
+    case 161: return launch_pack_inst<16, 1>(a, s);
+    case 321: return launch_pack_inst<32, 1>(a, s);
+    case 322: return launch_pack_inst<32, 2>(a, s);
+    default: return launch_pack_inst<32, 4>(a, s);
+    }
+}
+
+}  // namespace cplse

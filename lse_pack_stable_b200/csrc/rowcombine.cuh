@@ -1,0 +1,283 @@
+// Stable log-sum-exp merge of W partial attention outputs, one output row at a
+// time; shared by the fused pack->a2a->combine kernel and the combine kernel,
+// so that both produce the same bits for the same LSE values.
+//
+// Method (vLLM-Ascend pull request "Fuse local SFA LSE formation into DCP
+// pack", section "What this PR does / why we need it?"): each rank's
+// contribution carries LSE = softmax_max + log(softmax_sum), -inf when the
+// statistics are invalid; the stable combine merges the W contributions of a
+// row as LSE* = logsumexp_r LSE_r and O = sum_r exp(LSE_r - LSE*) O_r, with
+// -inf contributions weighted zero and an all-invalid row giving O = 0,
+// LSE* = -inf.
+//
+// Work split. A warp owns chunks of 32 consecutive output rows.
+//   Phase A: lane i takes row i of the chunk. It loads the row's W statistics
+//     (coalesced across the warp: consecutive rows are consecutive floats of
+//     each rank's plane), forms each LSE, and computes M, the sum, LSE* and the
+//     W weights sequentially in rank order, all in registers.
+//   Phase B: G lanes cover one row's D elements with 16-byte vectors (VPL per
+//     lane), 32/G rows per step. The row's weights and addresses reach the
+//     group by warp shuffles from the lane that owns the row. Every rank's
+//     vector is loaded before any is used (U steps at once), accumulated in
+//     fp32 in rank order, rounded to the payload type and stored.
+// An invalid contribution (weight 0) is neither loaded nor added: its payload
+// is replaced by -0.0, which leaves the fp32 accumulator (started at -0.0)
+// unchanged bit for bit.
+#pragma once
+
+#include <math.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace cplse {
+
+constexpr int kCombineThreads = 128;
+constexpr unsigned kFull = 0xffffffffu;
+constexpr uint32_t kNegZero2 = 0x80008000u;   // two -0.0 payload elements
+
+enum { kModeFused = 0, kModeCombine = 1 };
+
+// Phase A for one row: addresses and the W LSE values (-inf beyond W or q).
+template <int MODE, int WMAX>
+__device__ __forceinline__ void row_stats(const CombineArgs& a, int64_t q, bool qv,
+                                          int64_t& src_row, int64_t& dst_row, float (&lse)[WMAX])
+{
+    if (MODE == kModeFused) {
+        int64_t t = 0, h = 0;
+        if (qv) {
+            t = q / a.H;
+            h = q - t * a.H;
+        }
+        const int64_t j = h / a.Hc;
+        const int64_t hc = h - j * a.Hc;
+        src_row = t * a.so_t + h * a.so_h;
+        dst_row = (j * a.T + t) * a.Hc + hc;
+        const float* pm = a.smax + t * a.sm_t + h * a.sm_h;
+        const float* ps = a.ssum + t * a.ss_t + h * a.ss_h;
+        float m[WMAX], s[WMAX];
+#pragma unroll
+        for (int r = 0; r < WMAX; ++r) {
+            if (qv && r < a.W) {
+                m[r] = ld_stream(pm + r * a.sm_r);
+                s[r] = ld_stream(ps + r * a.ss_r);
+            } else {
+                m[r] = -INFINITY;
+                s[r] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < WMAX; ++r) {
+            // invalid statistic: non-finite max, non-finite sum, or sum <= 0
+            const bool ok = isfinite(m[r]) && isfinite(s[r]) && s[r] > 0.f;
+            lse[r] = ok ? m[r] + logf(s[r]) : -INFINITY;
+        }
+    } else {
+        int64_t j = 0, n = 0;
+        if (qv) {
+            j = q / a.N;
+            n = q - j * a.N;
+        }
+        src_row = (j * a.W * a.N + n) * a.D;
+        dst_row = q;
+        const float* pl = a.lse + j * a.W * a.N + n;
+#pragma unroll
+        for (int r = 0; r < WMAX; ++r) {
+            float x = (qv && r < a.W) ? ld_stream(pl + r * a.N) : -INFINITY;
+            lse[r] = x > -INFINITY ? x : -INFINITY;   // NaN counts as invalid
+        }
+    }
+}
+
+template <typename P, int MODE, int WMAX, int G, int VPL, int U>
+__global__ void __launch_bounds__(kCombineThreads)
+rowcombine_kernel(const CombineArgs a)
+{
+    constexpr int RPI = 32 / G;          // rows per step
+    constexpr int STEPS = 32 / RPI;      // steps per chunk
+    constexpr int RB = WMAX < 16 ? WMAX : 16;   // ranks loaded at once
+    static_assert(STEPS % U == 0, "U must divide the steps of a chunk");
+
+    const int lane = threadIdx.x & 31;
+    const int sub = lane / G;
+    const int gl = lane % G;
+    const int64_t warp = ((int64_t)blockIdx.x * kCombineThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * kCombineThreads) >> 5;
+    const int64_t nchunks = (a.rows + 31) >> 5;
+    const int V = a.D >> 3;
+    const int64_t rank_stride = a.rank_stride;
+
+    for (int64_t c = warp; c < nchunks; c += nwarps) {
+        // ---------------- phase A: lane owns row c*32 + lane
+        const int64_t q = c * 32 + lane;
+        const bool qv = q < a.rows;
+        int64_t src_row, dst_row;
+        float lse[WMAX];
+        row_stats<MODE, WMAX>(a, q, qv, src_row, dst_row, lse);
+
+        float M = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < WMAX; ++r) M = fmaxf(M, lse[r]);
+        float w[WMAX];
+        float L = -INFINITY;
+        if (M > -INFINITY) {
+            float S = 0.f;
+#pragma unroll
+            for (int r = 0; r < WMAX; ++r)
+                if (lse[r] > -INFINITY) S += expf(lse[r] - M);
+            L = M + logf(S);
+#pragma unroll
+            for (int r = 0; r < WMAX; ++r)
+                w[r] = lse[r] > -INFINITY ? expf(lse[r] - L) : 0.f;
+        } else {
+#pragma unroll
+            for (int r = 0; r < WMAX; ++r) w[r] = 0.f;
+        }
+        if (qv) st_stream(a.out_lse + dst_row, L);
+        const bool row_dead = !(M > -INFINITY);
+
+        // ---------------- phase B: G lanes per row
+#pragma unroll 1
+        for (int s0 = 0; s0 < STEPS; s0 += U) {
+            int64_t sb[U], db[U];
+            bool rv[U], dead[U];
+            float ws[U][WMAX];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int k = (s0 + u) * RPI + sub;
+                sb[u] = __shfl_sync(kFull, src_row, k);
+                db[u] = __shfl_sync(kFull, dst_row, k);
+                dead[u] = __shfl_sync(kFull, (int)row_dead, k) != 0;
+                rv[u] = c * 32 + k < a.rows;
+#pragma unroll
+                for (int r = 0; r < WMAX; ++r) ws[u][r] = __shfl_sync(kFull, w[r], k);
+            }
+            float acc[U][VPL][8];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int e = 0; e < VPL; ++e)
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) acc[u][e][x] = -0.f;
+
+#pragma unroll
+            for (int r0 = 0; r0 < WMAX; r0 += RB) {
+                uint4 v[U][VPL][RB];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+#pragma unroll
+                    for (int e = 0; e < VPL; ++e) {
+                        const int vec = gl + e * G;
+                        const uint4* base = reinterpret_cast<const uint4*>(a.src + sb[u]) + vec;
+#pragma unroll
+                        for (int rr = 0; rr < RB; ++rr) {
+                            const int r = r0 + rr;
+                            if (rv[u] && vec < V && ws[u][r] != 0.f)
+                                v[u][e][rr] = ld_stream(base + (r * rank_stride >> 3));
+                            else
+                                v[u][e][rr] = make_uint4(kNegZero2, kNegZero2, kNegZero2, kNegZero2);
+                        }
+                    }
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+#pragma unroll
+                    for (int e = 0; e < VPL; ++e)
+#pragma unroll
+                        for (int rr = 0; rr < RB; ++rr) {
+                            const float wr = ws[u][r0 + rr];
+                            const uint32_t wd[4] = {v[u][e][rr].x, v[u][e][rr].y, v[u][e][rr].z,
+                                                    v[u][e][rr].w};
+#pragma unroll
+                            for (int x = 0; x < 4; ++x) {
+                                const float2 f = unpack2<P>(wd[x]);
+                                acc[u][e][2 * x] = fmaf(wr, f.x, acc[u][e][2 * x]);
+                                acc[u][e][2 * x + 1] = fmaf(wr, f.y, acc[u][e][2 * x + 1]);
+                            }
+                        }
+            }
+
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int e = 0; e < VPL; ++e) {
+                    const int vec = gl + e * G;
+                    if (!(rv[u] && vec < V)) continue;
+                    uint4 o;
+                    if (dead[u]) {
+                        o = make_uint4(0u, 0u, 0u, 0u);   // all-invalid row: +0
+                    } else {
+                        o.x = pack2<P>(acc[u][e][0], acc[u][e][1]);
+                        o.y = pack2<P>(acc[u][e][2], acc[u][e][3]);
+                        o.z = pack2<P>(acc[u][e][4], acc[u][e][5]);
+                        o.w = pack2<P>(acc[u][e][6], acc[u][e][7]);
+                    }
+                    st_stream(reinterpret_cast<uint4*>(a.out + db[u] * a.D) + vec, o);
+                }
+        }
+    }
+}
+
+// Lanes per row and vectors per lane for a head dim of D elements (D % 8 == 0).
+struct RowShape {
+    int G, VPL;
+};
+
+inline RowShape row_shape(int D)
+{
+    const int V = D / kVecElems;
+    if (V <= 4) return {4, 1};
+    if (V <= 8) return {8, 1};
+    if (V <= 16) return {16, 1};
+    if (V <= 32) return {32, 1};
+    if (V <= 64) return {32, 2};
+    return {32, 4};
+}
+
+template <typename P, int MODE, int WMAX, int G, int VPL>
+cudaError_t launch_rowcombine_inst(const CombineArgs& a, cudaStream_t s)
+{
+    constexpr int U0 = (WMAX * VPL) >= 8 ? 1 : 8 / (WMAX * VPL);
+    constexpr int U = U0 > G ? G : U0;
+    auto kern = rowcombine_kernel<P, MODE, WMAX, G, VPL, U>;
+    static int per_sm = 0;
+    if (per_sm == 0) {
+        int n = 0;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kCombineThreads, 0);
+        if (e != cudaSuccess) return e;
+        per_sm = n > 0 ? n : 1;
+    }
+    const int64_t nchunks = (a.rows + 31) / 32;
+    const int64_t warps_per_block = kCombineThreads / 32;
+    int64_t blocks = (nchunks + warps_per_block - 1) / warps_per_block;
+    const int64_t cap = (int64_t)per_sm * sm_count();
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    kern<<<(unsigned)blocks, kCombineThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename P, int MODE, int WMAX>
+cudaError_t launch_rowcombine_w(const CombineArgs& a, cudaStream_t s)
+{
+    const RowShape rs = row_shape(a.D);
+    switch (rs.G * 10 + rs.VPL) {
+    case 41: return launch_rowcombine_inst<P, MODE, WMAX, 4, 1>(a, s);
+    case 81: return launch_rowcombine_inst<P, MODE, WMAX, 8, 1>(a, s);
+    case 161: return launch_rowcombine_inst<P, MODE, WMAX, 16, 1>(a, s);
+    case 321: return launch_rowcombine_inst<P, MODE, WMAX, 32, 1>(a, s);
+    case 322: return launch_rowcombine_inst<P, MODE, WMAX, 32, 2>(a, s);
+    default: return launch_rowcombine_inst<P, MODE, WMAX, 32, 4>(a, s);
+    }
+}
+
+template <typename P, int MODE>
+cudaError_t launch_rowcombine_p(const CombineArgs& a, cudaStream_t s)
+{
+    if (a.W <= 2) return launch_rowcombine_w<P, MODE, 2>(a, s);
+    if (a.W <= 4) return launch_rowcombine_w<P, MODE, 4>(a, s);
+    if (a.W <= 8) return launch_rowcombine_w<P, MODE, 8>(a, s);
+    if (a.W <= 16) return launch_rowcombine_w<P, MODE, 16>(a, s);
+    return launch_rowcombine_w<P, MODE, 32>(a, s);
+}
+
+}  // namespace cplse
