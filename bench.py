@@ -73,6 +73,23 @@ def config_block(wl: synth.Workload, world: int, extra=None):
     return c
 
 
+def reduce_max(values, world, device):
+    """Element-wise max of `values` over all ranks (the device time of a
+    multi-GPU step is the slowest rank's); identity on one rank."""
+    if world == 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world, bytes_per_step, steps, total_ms):
+    """Whole-job GB/s: every rank's bytes over the (max-over-ranks) time."""
+    return world * bytes_per_step * steps / (total_ms * 1e-3) / 1e9
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -334,12 +351,9 @@ def run_ours(args):
     total_ms = t_start.elapsed_time(t_end)
     launch_ms = [a.elapsed_time(b) for a, b in ev]
     mean_launch_ms = sum(launch_ms) / K
-    if world > 1:
-        t = torch.tensor([total_ms, mean_launch_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, mean_launch_ms = t.tolist()
+    total_ms, mean_launch_ms = reduce_max([total_ms, mean_launch_ms], world, dev)
     ms_per_step = total_ms / K
-    value = world * bytes_per_call * K / (total_ms * 1e-3) / 1e9
+    value = job_throughput(world, bytes_per_call, K, total_ms)
 
     peak, peak_kind = measured_peak()
     achieved = bytes_per_call / (mean_launch_ms * 1e-3) / 1e9
@@ -425,12 +439,8 @@ def measure_e2e(cp, wl, o_h, m_h, s_h, st, stream, dev, K, Wm, barrier, world, d
     b.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms = a.elapsed_time(b) / ke
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
-    return {"value": round(world * wl.fused_bytes() / (ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+    ms = reduce_max([a.elapsed_time(b) / ke], world, dev)[0]
+    return {"value": round(job_throughput(world, wl.fused_bytes(), 1, ms), 3), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4),
             "steps": ke, "note": "GB/s of the kernel's algorithmic bytes; the step is bound by "
                                  "the host link carrying h2d+d2h bytes"}

@@ -27,7 +27,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIBRARY_PATH = os.path.join(_HERE, "libcplse.so")
 
 if not os.path.exists(LIBRARY_PATH):
-    raise ImportError("libcplse.so is not built: run `python -m lse_pack_stable_b200.build` "
+    raise ImportError("libcplse.so is not built: run `python lse_pack_stable_b200/build.py` "
                       "(or __graft_entry__.build())")
 
 _lib = ctypes.CDLL(LIBRARY_PATH)

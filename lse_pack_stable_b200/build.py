@@ -1,6 +1,6 @@
 """Build libcplse.so (the CUDA kernels and the C-ABI) in-tree, for sm_100a only.
 
-    python -m lse_pack_stable_b200.build [--force] [-v]
+    python lse_pack_stable_b200/build.py [--force] [-v]
 
 Each csrc/*.cu compiles to an object in _build/ (in parallel), then nvcc links
 the shared library next to this file. The CUDA runtime is linked statically

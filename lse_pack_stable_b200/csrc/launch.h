@@ -29,6 +29,7 @@ struct CombineArgs {
     int64_t T;                // fused: tokens
     int64_t N;                // combine: rows per block
     int64_t rows;             // output rows
+    int dense_rows;           // fused: rank rows back to back (so_h == D, so_t == H*D)
 };
 
 struct PackArgs {
@@ -54,8 +55,12 @@ struct UlyssesArgs {
     int mode;                 // 0: seq->head, 1: head->seq
 };
 
+// register-staged merge (rowcombine.cuh)
 cudaError_t launch_fused(const CombineArgs& a, Dtype dt, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, Dtype dt, cudaStream_t s);
+// shared-memory-staged merge (rowcombine_async.cuh): same arithmetic, same bits
+cudaError_t launch_fused_async(const CombineArgs& a, Dtype dt, cudaStream_t s);
+cudaError_t launch_combine_async(const CombineArgs& a, Dtype dt, cudaStream_t s);
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t s);
 cudaError_t launch_permute(const void* send, void* recv, int W, int64_t block_bytes,
                            cudaStream_t s);

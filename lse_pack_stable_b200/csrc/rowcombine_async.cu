@@ -1,0 +1,93 @@
+// Shared-memory-staged stable log-sum-exp merge: launch planning for the
+// fused pack->a2a->combine and for the combine of a received packet.
+#include <type_traits>
+
+#include "rowcombine_async.cuh"
+
+namespace cplse {
+namespace {
+
+// Stages per warp: enough that about 16 KB of every warp's payload is in
+// flight (NST-1 slots), between 3 and 8.
+template <int WMAX, int VPL>
+constexpr int stages_for()
+{
+    constexpr int slot = VPL * WMAX * 32 * 16;
+    constexpr int n = 16384 / slot + 1;
+    return n < 3 ? 3 : (n > 8 ? 8 : n);
+}
+
+template <typename P, int MODE, int WMAX, int G, int VPL>
+cudaError_t launch_async_inst(const CombineArgs& a, cudaStream_t s)
+{
+    constexpr int NST = stages_for<WMAX, VPL>();
+    using Ring = AsyncRing<WMAX, VPL, NST>;
+    constexpr int smem = (kAsyncThreads / 32) * Ring::kWarpBytes;
+    auto kern = rowcombine_async_kernel<P, MODE, WMAX, G, VPL, NST>;
+    static int per_sm = 0;
+    if (per_sm == 0) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        int n = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kAsyncThreads, smem);
+        if (e != cudaSuccess) return e;
+        per_sm = n > 0 ? n : 1;
+    }
+    const int64_t nchunks = (a.rows + 31) / 32;
+    int64_t blocks = (nchunks + kAsyncThreads / 32 - 1) / (kAsyncThreads / 32);
+    const int64_t cap = (int64_t)per_sm * sm_count();
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    kern<<<(unsigned)blocks, kAsyncThreads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename P, int MODE, int WMAX, int G, int VPL>
+cudaError_t launch_staged(const CombineArgs& a, cudaStream_t s)
+{
+    // a ring that leaves fewer than one block per SM: register staging instead
+    constexpr int NST = stages_for<WMAX, VPL>();
+    constexpr int smem = (kAsyncThreads / 32) * AsyncRing<WMAX, VPL, NST>::kWarpBytes;
+    if (smem > 200 * 1024) return launch_rowcombine_inst<P, MODE, WMAX, G, VPL>(a, s);
+    return launch_async_inst<P, MODE, WMAX, G, VPL>(a, s);
+}
+
+template <typename P, int MODE, int WMAX>
+cudaError_t launch_async_w(const CombineArgs& a, cudaStream_t s)
+{
+    const RowShape rs = row_shape(a.D);
+    switch (rs.G * 10 + rs.VPL) {
+    case 41: return launch_staged<P, MODE, WMAX, 4, 1>(a, s);
+    case 81: return launch_staged<P, MODE, WMAX, 8, 1>(a, s);
+    case 161: return launch_staged<P, MODE, WMAX, 16, 1>(a, s);
+    case 321: return launch_staged<P, MODE, WMAX, 32, 1>(a, s);
+    case 322: return launch_staged<P, MODE, WMAX, 32, 2>(a, s);
+    default: return launch_staged<P, MODE, WMAX, 32, 4>(a, s);
+    }
+}
+
+template <typename P, int MODE>
+cudaError_t launch_async_p(const CombineArgs& a, cudaStream_t s)
+{
+    if (a.W <= 2) return launch_async_w<P, MODE, 2>(a, s);
+    if (a.W <= 4) return launch_async_w<P, MODE, 4>(a, s);
+    if (a.W <= 8) return launch_async_w<P, MODE, 8>(a, s);
+    if (a.W <= 16) return launch_async_w<P, MODE, 16>(a, s);
+    return launch_async_w<P, MODE, 32>(a, s);
+}
+
+}  // namespace
+
+cudaError_t launch_fused_async(const CombineArgs& a, Dtype dt, cudaStream_t s)
+{
+    return dt == Dtype::kBf16 ? launch_async_p<Bf16, kModeFused>(a, s)
+                              : launch_async_p<Fp16, kModeFused>(a, s);
+}
+
+cudaError_t launch_combine_async(const CombineArgs& a, Dtype dt, cudaStream_t s)
+{
+    return dt == Dtype::kBf16 ? launch_async_p<Bf16, kModeCombine>(a, s)
+                              : launch_async_p<Fp16, kModeCombine>(a, s);
+}
+
+}  // namespace cplse
