@@ -13,10 +13,12 @@
 // weights of the next chunk (phase A) and merges the current one (phase B).
 //
 // Work: warp w owns chunks w, w + nwarps, ... of 32 output rows; a chunk has
-// STEPS = G steps of RPI = 32/G rows. A "group" is one step of one chunk; group
-// number n of the warp is chunk n / STEPS, step n % STEPS. Group n lands in
-// ring slot n % NST. The first group of a chunk also brings the chunk's
-// statistics (lane = row) into the warp's statistics slot (chunk parity).
+// STEPS = G steps of RPI = 32/G rows. A "group" is one step of one chunk;
+// group number n of the warp is chunk n / STEPS, step n % STEPS (compile-time
+// divisors). Group n lands in ring slot n % NST. The first group of a chunk
+// also brings the chunk's statistics (lane = row) into statistics slot
+// chunk % NSTAT, where NSTAT = (NST-1)/STEPS + 1 guarantees the slot was read
+// (phase A of an older chunk) before it is refilled NST-1 groups ahead.
 // Every lane reads back only the 16-byte vectors it copied itself, so
 // cp.async.wait_group alone orders the copies before their use: there are no
 // barriers and no spin-waits.
@@ -30,7 +32,15 @@
 
 namespace cplse {
 
-constexpr int kAsyncThreads = 128;
+#ifndef CPLSE_ASYNC_THREADS
+#define CPLSE_ASYNC_THREADS 128
+#endif
+#ifndef CPLSE_ASYNC_INFLIGHT
+#define CPLSE_ASYNC_INFLIGHT 4096
+#endif
+constexpr int kAsyncThreads = CPLSE_ASYNC_THREADS;
+// payload bytes each warp keeps in flight (sets the ring depth NST)
+constexpr int kAsyncInflight = CPLSE_ASYNC_INFLIGHT;
 
 __device__ __forceinline__ uint32_t sh_addr(const void* p)
 {
@@ -90,112 +100,143 @@ __device__ __forceinline__ void row_addr(const CombineArgs& a, int64_t q, int64_
 }
 
 // Shared memory per warp: NST payload slots of [VPL][WMAX][32 lanes] 16-byte
-// vectors, then two statistics slots of [2][WMAX][32] floats.
-template <int WMAX, int VPL, int NST>
+// vectors; NSTAT statistics slots of [2][WMAX][32] floats; and the chunk's row
+// table: weights [32][WS] (WS = WMAX rounded up to 4, for 16-byte reads) and
+// destination rows [32] (bitwise-complemented for an all-invalid row).
+template <int WMAX, int G, int VPL, int NST>
 struct AsyncRing {
     static constexpr int kSlotVecs = VPL * WMAX * 32;
     static constexpr int kPayBytes = NST * kSlotVecs * 16;
-    static constexpr int kStatBytes = 2 * 2 * WMAX * 32 * 4;
-    static constexpr int kWarpBytes = kPayBytes + kStatBytes;
+    static constexpr int kStatSlotFloats = 2 * WMAX * 32;
+    static constexpr int kStat = (NST - 1) / G + 1;
+    static constexpr int kStatBytes = kStat * kStatSlotFloats * 4;
+    static constexpr int WS = (WMAX + 3) / 4 * 4;
+    static constexpr int kTabBytes = 32 * WS * 4 + 32 * 8;
+    static constexpr int kWarpBytes = kPayBytes + kStatBytes + kTabBytes;
 };
 
 template <typename P, int MODE, int WMAX, int G, int VPL, int NST>
 __global__ void __launch_bounds__(kAsyncThreads)
 rowcombine_async_kernel(const CombineArgs a)
 {
-    using Ring = AsyncRing<WMAX, VPL, NST>;
+    using Ring = AsyncRing<WMAX, G, VPL, NST>;
     constexpr int RPI = 32 / G;
     constexpr int STEPS = G;
+    constexpr int WS = Ring::WS;
     extern __shared__ __align__(16) uint8_t smem[];
     const int lane = threadIdx.x & 31;
     const int wib = threadIdx.x >> 5;
-    uint4* ring = reinterpret_cast<uint4*>(smem + wib * Ring::kWarpBytes);
-    float* sring = reinterpret_cast<float*>(smem + wib * Ring::kWarpBytes + Ring::kPayBytes);
+    uint8_t* wbase = smem + wib * Ring::kWarpBytes;
+    uint4* ring = reinterpret_cast<uint4*>(wbase);
+    float* sring = reinterpret_cast<float*>(wbase + Ring::kPayBytes);
+    float* wtab = reinterpret_cast<float*>(wbase + Ring::kPayBytes + Ring::kStatBytes);
+    int64_t* dtab = reinterpret_cast<int64_t*>(wbase + Ring::kPayBytes + Ring::kStatBytes + 32 * WS * 4);
     const int sub = lane / G;
     const int gl = lane % G;
     const int V = a.D >> 3;
     const int W = a.W;
+    const int64_t rs16 = a.rank_stride >> 3;              // rank stride in 16-byte vectors
+    const uint4* src16 = reinterpret_cast<const uint4*>(a.src);
     const int64_t warp = ((int64_t)blockIdx.x * kAsyncThreads + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * kAsyncThreads) >> 5;
     const int64_t nchunks = (a.rows + 31) >> 5;
     const int64_t my_chunks = warp < nchunks ? (nchunks - warp + nwarps - 1) / nwarps : 0;
     const int64_t ngroups = my_chunks * STEPS;
 
-    // enqueue the copies of group n (an empty group past the end)
-    auto issue = [&](int64_t n) {
-        if (n < ngroups) {
-            const int64_t ci = n / STEPS;
-            const int step = (int)(n - ci * STEPS);
-            const int64_t c = warp + ci * nwarps;
-            const int slot = (int)(n % NST);
-            if (step == 0) {   // this chunk's statistics, lane = row
+    // payload vector offset (rank 0) of output row q
+    auto row_src = [&](int64_t q) -> int64_t {
+        if (MODE == kModeFused) {
+            if (a.dense_rows) return q * (a.D >> 3);
+            int64_t t, h;
+            divmod_u(q, a.H, t, h);
+            return (t * a.so_t + h * a.so_h) >> 3;
+        } else {
+            int64_t j, n;
+            divmod_u(q, a.N, j, n);
+            return ((j * W * a.N + n) * a.D) >> 3;
+        }
+    };
+
+    // issue cursor: group ni = chunk ci_i, step st_i, ring slot sl_i
+    int64_t ni = 0, ci_i = 0;
+    int st_i = 0, sl_i = 0;
+    auto issue_next = [&]() {
+        if (ni < ngroups) {
+            const int64_t c = warp + ci_i * nwarps;
+            if (st_i == 0) {   // this chunk's statistics, lane = row
                 const int64_t q = c * 32 + lane;
                 if (q < a.rows) {
-                    float* sl = sring + (int)(ci & 1) * (2 * WMAX * 32);
+                    float* sl = sring + (int)(ci_i % Ring::kStat) * Ring::kStatSlotFloats;
                     if (MODE == kModeFused) {
                         int64_t t, h;
                         divmod_u(q, a.H, t, h);
+                        const float* pm = a.smax + t * a.sm_t + h * a.sm_h;
+                        const float* ps = a.ssum + t * a.ss_t + h * a.ss_h;
 #pragma unroll
                         for (int r = 0; r < WMAX; ++r)
                             if (r < W) {
-                                cp_async_f32(sh_addr(sl + r * 32 + lane),
-                                             a.smax + r * a.sm_r + t * a.sm_t + h * a.sm_h);
-                                cp_async_f32(sh_addr(sl + (WMAX + r) * 32 + lane),
-                                             a.ssum + r * a.ss_r + t * a.ss_t + h * a.ss_h);
+                                cp_async_f32(sh_addr(sl + r * 32 + lane), pm + r * a.sm_r);
+                                cp_async_f32(sh_addr(sl + (WMAX + r) * 32 + lane), ps + r * a.ss_r);
                             }
                     } else {
                         int64_t j, nn;
                         divmod_u(q, a.N, j, nn);
+                        const float* pl = a.lse + j * W * a.N + nn;
 #pragma unroll
                         for (int r = 0; r < WMAX; ++r)
-                            if (r < W)
-                                cp_async_f32(sh_addr(sl + r * 32 + lane),
-                                             a.lse + (j * W + r) * a.N + nn);
+                            if (r < W) cp_async_f32(sh_addr(sl + r * 32 + lane), pl + r * a.N);
                     }
                 }
             }
-            const int64_t q = c * 32 + step * RPI + sub;
+            const int64_t q = c * 32 + st_i * RPI + sub;
             if (q < a.rows) {
-                int64_t src, dst;
-                row_addr<MODE>(a, q, src, dst);
-                const uint4* base = reinterpret_cast<const uint4*>(a.src + src);
-                uint4* sl = ring + slot * Ring::kSlotVecs;
+                const uint4* base = src16 + row_src(q) + gl;
+                uint4* sl = ring + sl_i * Ring::kSlotVecs + lane;
 #pragma unroll
                 for (int e = 0; e < VPL; ++e) {
-                    const int vec = gl + e * G;
-                    if (vec < V) {
+                    if (gl + e * G < V) {
 #pragma unroll
                         for (int r = 0; r < WMAX; ++r)
-                            if (r < W)
-                                cp_async16(sh_addr(sl + (e * WMAX + r) * 32 + lane),
-                                           base + vec + ((r * a.rank_stride) >> 3));
+                            if (r < W) cp_async16(sh_addr(sl + (e * WMAX + r) * 32), base + e * G + r * rs16);
                     }
                 }
             }
+            ++ni;
+            if (++st_i == STEPS) {
+                st_i = 0;
+                ++ci_i;
+            }
+            if (++sl_i == NST) sl_i = 0;
         }
         cp_async_commit();
     };
 
     // prologue: NST-1 groups in flight
-#pragma unroll
-    for (int d = 0; d < NST - 1; ++d) issue(d);
+#pragma unroll 1
+    for (int d = 0; d < NST - 1; ++d) issue_next();
 
-    float w[WMAX];
-    int64_t dst_own = 0;
-    bool dead_own = true;
+    int64_t ci = 0;
+    int step = 0, slot = 0;
     for (int64_t n = 0; n < ngroups; ++n) {
         cp_async_wait<NST - 2>();       // group n has landed (this lane's copies)
-        issue(n + NST - 1);             // refill the slot that group n-1 used
-        const int64_t ci = n / STEPS;
-        const int step = (int)(n - ci * STEPS);
+        issue_next();                   // refill the slot that group n-1 used
         const int64_t c = warp + ci * nwarps;
         if (step == 0) {
             // ---------------- phase A: lane owns row c*32 + lane
             const int64_t q = c * 32 + lane;
             const bool qv = q < a.rows;
-            int64_t src_unused = 0;
-            if (qv) row_addr<MODE>(a, q, src_unused, dst_own);
-            const float* sl = sring + (int)(ci & 1) * (2 * WMAX * 32);
+            int64_t dst = 0;
+            if (qv) {
+                if (MODE == kModeFused) {
+                    int64_t t, h, j, hc;
+                    divmod_u(q, a.H, t, h);
+                    divmod_u(h, a.Hc, j, hc);
+                    dst = (j * a.T + t) * a.Hc + hc;
+                } else {
+                    dst = q;
+                }
+            }
+            const float* sl = sring + (int)(ci % Ring::kStat) * Ring::kStatSlotFloats;
             float lse[WMAX];
 #pragma unroll
             for (int r = 0; r < WMAX; ++r) {
@@ -216,6 +257,9 @@ rowcombine_async_kernel(const CombineArgs a)
 #pragma unroll
             for (int r = 0; r < WMAX; ++r) M = fmaxf(M, lse[r]);
             float L = -INFINITY;
+            float w[WS];
+#pragma unroll
+            for (int r = 0; r < WS; ++r) w[r] = 0.f;
             if (M > -INFINITY) {
                 float S = 0.f;
 #pragma unroll
@@ -224,23 +268,33 @@ rowcombine_async_kernel(const CombineArgs a)
                 L = M + logf(S);
 #pragma unroll
                 for (int r = 0; r < WMAX; ++r) w[r] = lse[r] > -INFINITY ? expf(lse[r] - L) : 0.f;
-            } else {
-#pragma unroll
-                for (int r = 0; r < WMAX; ++r) w[r] = 0.f;
             }
-            if (qv) st_stream(a.out_lse + dst_own, L);
-            dead_own = !(M > -INFINITY);
+            if (qv) st_stream(a.out_lse + dst, L);
+            __syncwarp();                                   // the previous chunk's table is read
+#pragma unroll
+            for (int r = 0; r < WS; r += 4)
+                *reinterpret_cast<float4*>(wtab + lane * WS + r) =
+                    make_float4(w[r], w[r + 1], w[r + 2], w[r + 3]);
+            dtab[lane] = (M > -INFINITY) ? dst : ~dst;
+            __syncwarp();                                   // the table is visible to the warp
         }
         // ---------------- phase B: this step's RPI rows, G lanes per row
-        const int k = step * RPI + sub;                       // row of the chunk
+        const int k = step * RPI + sub;                     // row of the chunk
         const int64_t q = c * 32 + k;
-        const int64_t db = __shfl_sync(kFull, dst_own, k);
-        const bool dead = __shfl_sync(kFull, (int)dead_own, k) != 0;
-        float ws[WMAX];
-#pragma unroll
-        for (int r = 0; r < WMAX; ++r) ws[r] = __shfl_sync(kFull, w[r], k);
         if (q < a.rows) {
-            const uint4* sl = ring + (int)(n % NST) * Ring::kSlotVecs;
+            int64_t db = dtab[k];
+            const bool dead = db < 0;
+            if (dead) db = ~db;
+            float ws[WS];
+#pragma unroll
+            for (int r = 0; r < WS; r += 4) {
+                const float4 f = *reinterpret_cast<const float4*>(wtab + k * WS + r);
+                ws[r] = f.x;
+                ws[r + 1] = f.y;
+                ws[r + 2] = f.z;
+                ws[r + 3] = f.w;
+            }
+            const uint4* sl = ring + slot * Ring::kSlotVecs + lane;
 #pragma unroll
             for (int e = 0; e < VPL; ++e) {
                 const int vec = gl + e * G;
@@ -251,7 +305,7 @@ rowcombine_async_kernel(const CombineArgs a)
 #pragma unroll
                 for (int r = 0; r < WMAX; ++r) {
                     if (r >= W) break;
-                    uint4 v = sl[(e * WMAX + r) * 32 + lane];
+                    uint4 v = sl[(e * WMAX + r) * 32];
                     if (!(ws[r] != 0.f)) v = make_uint4(kNegZero2, kNegZero2, kNegZero2, kNegZero2);
                     const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -273,6 +327,11 @@ rowcombine_async_kernel(const CombineArgs a)
                 st_stream(reinterpret_cast<uint4*>(a.out + db * a.D) + vec, o);
             }
         }
+        if (++step == STEPS) {
+            step = 0;
+            ++ci;
+        }
+        if (++slot == NST) slot = 0;
     }
     cp_async_wait<0>();
 }
