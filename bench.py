@@ -40,8 +40,9 @@ import synth  # noqa: E402
 
 METRIC = "pack+permute+combine µs/call and effective HBM GB/s (% of B200 peak)"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["lse_pack_stable_b200/csrc/rowcombine.cuh", "lse_pack_stable_b200/csrc/fused.cu",
-                  "lse_pack_stable_b200/csrc/common.cuh"]
+KERNEL_SOURCES = ["lse_pack_stable_b200/csrc/rowcombine_async.cuh",
+                  "lse_pack_stable_b200/csrc/rowcombine_async.cu",
+                  "lse_pack_stable_b200/csrc/rowcombine.cuh", "lse_pack_stable_b200/csrc/common.cuh"]
 
 
 def parse():
@@ -288,18 +289,28 @@ def run_ours(args):
     W, T, H, D, Hc = wl.W, wl.T, wl.H, wl.D, wl.Hc
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float16
 
-    # ---- inputs (host generation, then upload); rotate sets so every step reads cold HBM
-    o_h, m_h, s_h = sample_inputs(wl, T) if W * T * H * D <= (1 << 31) else (None, None, None)
-    if o_h is None:
-        raise SystemExit("workload too large for the host-generated benchmark inputs")
-    in_bytes = o_h.nbytes + m_h.nbytes + s_h.nbytes
+    # ---- inputs: generated on the host block by block into pinned memory (the
+    # end-to-end leg copies from there), uploaded once; extra device copies
+    # rotate so that every step reads cold HBM
+    o_h = torch.empty((W, T, H, D), dtype=torch.int16, pin_memory=True)
+    m_h = torch.empty((W, T, H), dtype=torch.float32, pin_memory=True)
+    s_h = torch.empty((W, T, H), dtype=torch.float32, pin_memory=True)
+    tb = max(1, (256 << 20) // (H * D * 2))
+    for r in range(W):
+        for t0 in range(0, T, tb):
+            t1 = min(T, t0 + tb)
+            o_h[r, t0:t1].numpy()[...] = synth.o_block(wl, r, t0, t1).view(np.int16)
+        mr, sr = synth.stats_block(wl, r)
+        m_h[r].numpy()[...] = mr
+        s_h[r].numpy()[...] = sr
+    in_bytes = o_h.numel() * 2 + m_h.numel() * 4 + s_h.numel() * 4
     out_bytes = T * H * D * 2 + T * H * 4
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     nsets = max(2, math.ceil(3 * l2 / (in_bytes + out_bytes)) + 1)
     nsets = min(nsets, max(2, int(40e9 // (in_bytes + out_bytes))))
-    o_d = torch.from_numpy(o_h.view(np.int16)).to(dev).view(tdt)
-    m_d = torch.from_numpy(m_h).to(dev)
-    s_d = torch.from_numpy(s_h).to(dev)
+    o_d = o_h.to(dev).view(tdt)
+    m_d = m_h.to(dev)
+    s_d = s_h.to(dev)
     sets = []
     for i in range(nsets):
         oi = o_d if i == 0 else o_d.clone()
@@ -360,7 +371,8 @@ def run_ours(args):
     roofline = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": recorded_traffic(args.config),
                 "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                else "fallback 6.65 TB/s", "kernel": "rowcombine_kernel (fused)",
+                else "fallback 6.65 TB/s", "kernel": ("rowcombine_kernel (register-staged, fused mode)" if W >= 16
+                           else "rowcombine_async_kernel (shared-memory-staged, fused mode)"),
                 "algorithmic_bytes_per_launch": bytes_per_call,
                 "us_per_launch": round(mean_launch_ms * 1e3, 3),
                 "us_per_launch_p10_p50_p90": [round(1e3 * np.percentile(launch_ms, q), 3)
@@ -378,7 +390,8 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, _, sample, cores = time_oracle(wl, 12.0, o_h, m_h, s_h)
+        gbs, _, sample, cores = time_oracle(wl, 12.0, o_h.numpy().view(np.uint16), m_h.numpy(),
+                                            s_h.numpy())
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                "sample": sample}
 
@@ -408,9 +421,7 @@ def measure_e2e(cp, wl, o_h, m_h, s_h, st, stream, dev, K, Wm, barrier, world, d
     pinned memory, the C-ABI call, and device->host copies of its outputs."""
     import torch
     oi, mi, si, out, ol = st
-    po = torch.from_numpy(o_h.view(np.int16)).pin_memory()
-    pm = torch.from_numpy(m_h).pin_memory()
-    ps = torch.from_numpy(s_h).pin_memory()
+    po, pm, ps = o_h, m_h, s_h
     ho = torch.empty(out.shape, dtype=torch.int16).pin_memory()
     hl = torch.empty(ol.shape, dtype=torch.float32).pin_memory()
     oi16 = oi.view(torch.int16)
@@ -469,9 +480,11 @@ def measure_breakdown(cp, wl, sets, stream, dev, peak, tdt):
     import torch
     W, T, H, D, Hc = wl.W, wl.T, wl.H, wl.D, wl.Hc
     n = len(sets)
+    # two packet buffers alternate (L2 rotation) unless one alone exceeds L2 many times
+    nb = 2 if W * T * H * D * 2 < 2e9 else 1
     pk = [(torch.empty((W, W, T, Hc, D), dtype=tdt, device=dev),
-           torch.empty((W, W, T, Hc), dtype=torch.float32, device=dev)) for _ in range(2)]
-    rv = [(torch.empty_like(pk[0][0]), torch.empty_like(pk[0][1])) for _ in range(2)]
+           torch.empty((W, W, T, Hc), dtype=torch.float32, device=dev)) for _ in range(nb)]
+    rv = [(torch.empty_like(pk[0][0]), torch.empty_like(pk[0][1])) for _ in range(nb)]
     res = {}
 
     def rec(name, ms, nbytes):
@@ -479,19 +492,19 @@ def measure_breakdown(cp, wl, sets, stream, dev, peak, tdt):
         res[name] = {"us": round(ms * 1e3, 2), "bytes": nbytes, "GB/s": round(gbs, 1),
                      "frac": round(gbs / peak, 4)}
 
-    rec("pack", _time(lambda i: cp.cp_pack_lse(*sets[i % n][:3], pkt_o=pk[i % 2][0],
-                                               pkt_lse=pk[i % 2][1], stream=stream), stream),
+    rec("pack", _time(lambda i: cp.cp_pack_lse(*sets[i % n][:3], pkt_o=pk[i % nb][0],
+                                               pkt_lse=pk[i % nb][1], stream=stream), stream),
         wl.pack_bytes())
     rows = W * T * H
 
     def perm(i):
-        cp.cp_a2a_local_permute(pk[i % 2][0], W, recv=rv[i % 2][0], stream=stream)
-        cp.cp_a2a_local_permute(pk[i % 2][1], W, recv=rv[i % 2][1], stream=stream)
+        cp.cp_a2a_local_permute(pk[i % nb][0], W, recv=rv[i % nb][0], stream=stream)
+        cp.cp_a2a_local_permute(pk[i % nb][1], W, recv=rv[i % nb][1], stream=stream)
     rec("permute", _time(perm, stream), 2 * rows * (D * 2 + 4))
     outs = [(torch.empty((W, T, Hc, D), dtype=tdt, device=dev),
-             torch.empty((W, T, Hc), dtype=torch.float32, device=dev)) for _ in range(2)]
-    rec("combine", _time(lambda i: cp.cp_lse_combine(*rv[i % 2], out=outs[i % 2][0],
-                                                     out_lse=outs[i % 2][1], stream=stream),
+             torch.empty((W, T, Hc), dtype=torch.float32, device=dev)) for _ in range(nb)]
+    rec("combine", _time(lambda i: cp.cp_lse_combine(*rv[i % nb], out=outs[i % nb][0],
+                                                     out_lse=outs[i % nb][1], stream=stream),
                          stream), wl.combine_bytes())
     unfused_us = res["pack"]["us"] + res["permute"]["us"] + res["combine"]["us"]
     res["unfused_total_us"] = round(unfused_us, 2)
