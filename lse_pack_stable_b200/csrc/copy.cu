@@ -22,6 +22,9 @@ template <typename V>
 __device__ __forceinline__ void st_cs(V* p, V v) { __stcs(p, v); }
 
 // recv[j][r] = send[r][j]; grid.y enumerates destination blocks d = j*W + r.
+// Each thread moves U vectors, U loads in flight before the first store; the
+// grid covers every vector once (no grid-stride loop), so blocks retire and
+// new ones start continuously instead of marching in lockstep.
 template <typename V, int U>
 __global__ void __launch_bounds__(kCopyThreads)
 permute_kernel(const V* __restrict__ send, V* __restrict__ recv, int W, int64_t nvec)
@@ -30,20 +33,17 @@ permute_kernel(const V* __restrict__ send, V* __restrict__ recv, int W, int64_t 
     const int j = d / W, r = d - j * W;
     const V* src = send + (int64_t)(r * W + j) * nvec;
     V* dst = recv + (int64_t)d * nvec;
-    const int64_t stride = (int64_t)gridDim.x * kCopyThreads * U;
-    for (int64_t base = (int64_t)blockIdx.x * kCopyThreads * U + threadIdx.x; base < nvec;
-         base += stride) {
-        V v[U];
+    const int64_t base = (int64_t)blockIdx.x * kCopyThreads * U + threadIdx.x;
+    V v[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t i = base + (int64_t)u * kCopyThreads;
-            if (i < nvec) v[u] = ld_cs(src + i);
-        }
+    for (int u = 0; u < U; ++u) {
+        const int64_t i = base + (int64_t)u * kCopyThreads;
+        if (i < nvec) v[u] = ld_cs(src + i);
+    }
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t i = base + (int64_t)u * kCopyThreads;
-            if (i < nvec) st_cs(dst + i, v[u]);
-        }
+    for (int u = 0; u < U; ++u) {
+        const int64_t i = base + (int64_t)u * kCopyThreads;
+        if (i < nvec) st_cs(dst + i, v[u]);
     }
 }
 
@@ -51,64 +51,84 @@ template <typename V>
 cudaError_t launch_permute_v(const void* send, void* recv, int W, int64_t block_bytes,
                              cudaStream_t s)
 {
-    constexpr int U = 4;
+    constexpr int U = 8;
     const int64_t nvec = block_bytes / (int64_t)sizeof(V);
-    int64_t gx = (nvec + kCopyThreads * U - 1) / (kCopyThreads * U);
-    // enough CTAs to fill every SM several times over; the rest is grid-stride
-    const int64_t want = (int64_t)sm_count() * 16;
-    const int64_t per_block_cap = (want + (int64_t)W * W - 1) / ((int64_t)W * W);
-    if (gx > per_block_cap) gx = per_block_cap;
-    if (gx < 1) gx = 1;
+    const int64_t gx = (nvec + kCopyThreads * U - 1) / (kCopyThreads * U);
+    if (gx > 0x7fffffff) return cudaErrorInvalidConfiguration;
     dim3 grid((unsigned)gx, (unsigned)(W * W));
     permute_kernel<V, U><<<grid, kCopyThreads, 0, s>>>(static_cast<const V*>(send),
                                                       static_cast<V*>(recv), W, nvec);
     return cudaGetLastError();
 }
 
-// One warp per contiguous chunk of Hc*D elements.
+// One warp per contiguous chunk of Hc*D elements, K chunks per iteration (all
+// their loads in flight before the first store).
 //   mode 0 (seq->head): chunk c = ((r*B + b)*S_l + s)*W + j of the input
 //       lands at chunk (j*B + b)*S + r*S_l + s of the output;
 //   mode 1 (head->seq): chunk c = (r*B + b)*S + (j*S_l + s) of the input
 //       lands at chunk ((j*B + b)*S_l + s)*W + r of the output.
-template <typename V, int MODE, int UNR>
+// x / d and x % d, on the 32-bit path when both operands fit.
+__device__ __forceinline__ int64_t div_u(int64_t x, int64_t d, int64_t& rem)
+{
+    if (((uint64_t)x | (uint64_t)d) < (1ull << 32)) {
+        const uint32_t q = (uint32_t)x / (uint32_t)d;
+        rem = (uint32_t)x - q * (uint32_t)d;
+        return q;
+    }
+    const int64_t q = x / d;
+    rem = x - q * d;
+    return q;
+}
+
+template <int MODE>
+__device__ __forceinline__ int64_t ulysses_dst_chunk(const UlyssesArgs& a, int64_t c)
+{
+    int64_t j, s, b, sg;
+    if (MODE == 0) {
+        int64_t rest = div_u(c, a.W, j);
+        rest = div_u(rest, a.S_l, s);
+        const int64_t r = div_u(rest, a.B, b);
+        return (j * a.B + b) * a.S + r * a.S_l + s;
+    }
+    const int64_t rest = div_u(c, a.S, sg);
+    const int64_t r = div_u(rest, a.B, b);
+    j = div_u(sg, a.S_l, s);
+    return ((j * a.B + b) * a.S_l + s) * a.W + r;
+}
+
+template <typename V, int MODE, int K, int UNR>
 __global__ void __launch_bounds__(kCopyThreads)
 ulysses_kernel(const V* __restrict__ in, V* __restrict__ out, const UlyssesArgs a, int64_t cv)
 {
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * kCopyThreads + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * kCopyThreads) >> 5;
-    for (int64_t c = warp; c < a.nchunks; c += nwarps) {
-        int64_t dc;
-        if (MODE == 0) {
-            int64_t rest = c / a.W;
-            const int64_t j = c - rest * a.W;
-            const int64_t s = rest % a.S_l;
-            rest /= a.S_l;
-            const int64_t b = rest % a.B;
-            const int64_t r = rest / a.B;
-            dc = (j * a.B + b) * a.S + r * a.S_l + s;
-        } else {
-            int64_t rest = c / a.S;
-            const int64_t sg = c - rest * a.S;
-            const int64_t b = rest % a.B;
-            const int64_t r = rest / a.B;
-            const int64_t j = sg / a.S_l;
-            const int64_t s = sg - j * a.S_l;
-            dc = ((j * a.B + b) * a.S_l + s) * a.W + r;
-        }
-        const V* src = in + c * cv;
-        V* dst = out + dc * cv;
-        for (int64_t v0 = lane; v0 < cv; v0 += 32 * UNR) {
-            V x[UNR];
+    for (int64_t c0 = warp; c0 < a.nchunks; c0 += nwarps * K) {
+        int64_t dcs[K];
 #pragma unroll
-            for (int u = 0; u < UNR; ++u) {
-                const int64_t i = v0 + 32 * u;
-                if (i < cv) x[u] = ld_cs(src + i);
+        for (int k = 0; k < K; ++k) {
+            const int64_t c = c0 + k * nwarps;
+            dcs[k] = c < a.nchunks ? ulysses_dst_chunk<MODE>(a, c) : 0;
+        }
+        for (int64_t v0 = lane; v0 < cv; v0 += 32 * UNR) {
+            V x[K][UNR];
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+                const int64_t c = c0 + k * nwarps;
+#pragma unroll
+                for (int u = 0; u < UNR; ++u) {
+                    const int64_t i = v0 + 32 * u;
+                    if (c < a.nchunks && i < cv) x[k][u] = ld_cs(in + c * cv + i);
+                }
             }
 #pragma unroll
-            for (int u = 0; u < UNR; ++u) {
-                const int64_t i = v0 + 32 * u;
-                if (i < cv) st_cs(dst + i, x[u]);
+            for (int k = 0; k < K; ++k) {
+                const int64_t c = c0 + k * nwarps;
+#pragma unroll
+                for (int u = 0; u < UNR; ++u) {
+                    const int64_t i = v0 + 32 * u;
+                    if (c < a.nchunks && i < cv) st_cs(out + dcs[k] * cv + i, x[k][u]);
+                }
             }
         }
     }
@@ -118,7 +138,8 @@ template <typename V, int MODE>
 cudaError_t launch_ulysses_v(const UlyssesArgs& a, cudaStream_t s)
 {
     constexpr int UNR = 4;
-    auto kern = ulysses_kernel<V, MODE, UNR>;
+    constexpr int K = 2;
+    auto kern = ulysses_kernel<V, MODE, K, UNR>;
     static int per_sm = 0;
     if (per_sm == 0) {
         int n = 0;

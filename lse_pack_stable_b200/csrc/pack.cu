@@ -23,6 +23,19 @@ namespace {
 
 constexpr int kPackThreads = 128;
 
+// 64-bit quotient and remainder, on the 32-bit path when both operands fit.
+__device__ __forceinline__ void divmod_pack(int64_t x, int64_t d, int64_t& q, int64_t& r)
+{
+    if (((uint64_t)x | (uint64_t)d) < (1ull << 32)) {
+        const uint32_t q32 = (uint32_t)x / (uint32_t)d;
+        q = q32;
+        r = (uint32_t)x - q32 * (uint32_t)d;
+    } else {
+        q = x / d;
+        r = x - q * d;
+    }
+}
+
 template <int G, int VPL, int U>
 __global__ void __launch_bounds__(kPackThreads) pack_kernel(const PackArgs a)
 {
@@ -45,17 +58,17 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const PackArgs a)
         const bool qv = q < a.rows;
         int64_t src_row = 0, dst_row = 0;
         if (qv) {
-            const int64_t r = q / TH;
-            const int64_t rem = q - r * TH;
-            const int64_t t = rem / a.H;
-            const int64_t h = rem - t * a.H;
+            int64_t r, rem, t, h;
+            divmod_pack(q, TH, r, rem);
+            divmod_pack(rem, (int64_t)a.H, t, h);
             int64_t j, slot;
             if (a.scatter_dim == 1) {
-                j = h / a.Hc;
-                slot = t * a.Hc + (h - j * a.Hc);
+                divmod_pack(h, (int64_t)a.Hc, j, slot);
+                slot += t * a.Hc;
             } else {
-                j = t / a.Tc;
-                slot = (t - j * a.Tc) * a.H + h;
+                int64_t tc;
+                divmod_pack(t, a.Tc, j, tc);
+                slot = tc * a.H + h;
             }
             dst_row = (r * a.W + j) * block_rows + slot;
             src_row = r * a.so_r + t * a.so_t + h * a.so_h;
@@ -93,6 +106,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const PackArgs a)
                         st_stream(reinterpret_cast<uint4*>(a.pkt_o + db[u] * a.D) + vec, v[u][e]);
                 }
         }
+
     }
 }
 
