@@ -496,6 +496,17 @@ def measure_breakdown(cp, wl, sets, stream, dev, peak, tdt):
                                                pkt_lse=pk[i % nb][1], stream=stream), stream),
         wl.pack_bytes())
     rows = W * T * H
+    # the Before pipeline of the DCP pull request: materialize LSE, then pack from it
+    lse_buf = torch.empty((W, T, H), dtype=torch.float32, device=dev)
+
+    def legacy(i):
+        oi, mi, si = sets[i % n][:3]
+        cp.cp_lse_materialize(mi, si, lse=lse_buf, stream=stream)
+        cp.cp_pack_from_lse(oi, lse_buf, pkt_o=pk[i % nb][0], pkt_lse=pk[i % nb][1], stream=stream)
+    legacy_bytes = rows * (8 + 4) + rows * (2 * D * 2 + 4 + 4)
+    rec("legacy_pack", _time(legacy, stream), legacy_bytes)
+    res["legacy_over_pack"] = round(res["legacy_pack"]["us"] / res["pack"]["us"], 3)
+    del lse_buf
 
     def perm(i):
         cp.cp_a2a_local_permute(pk[i % nb][0], W, recv=rv[i % nb][0], stream=stream)

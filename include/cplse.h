@@ -106,6 +106,29 @@ CPLSE_API cp_status cp_pack_lse(const void* o, cp_strides3 so, const float* smax
                       cp_dtype dt, int scatter_dim, void* pkt_o, float* pkt_lse, void* stream);
 
 /*
+ * [DCP] Before pipeline, first step ("materialize LSE = softmax_max +
+ * log(softmax_sum)"): the legacy path the pull request keeps for compatibility
+ * and regression coverage, here the A/B baseline of the max/sum-aware pack.
+ * Writes a standalone fp32 tensor lse [W][T][H] (contiguous) with the same
+ * values cp_pack_lse forms (max + logf(sum), -inf for invalid statistics).
+ *   smax, ssum fp32 [W][T][H], element strides sm / ss (>= 0).
+ */
+CPLSE_API cp_status cp_lse_materialize(const float* smax, cp_strides3 sm, const float* ssum,
+                                       cp_strides3 ss, int W, int64_t T, int H, float* lse,
+                                       void* stream);
+
+/*
+ * [DCP] Before pipeline, remaining steps ("permute / reshape", "DCP pack"):
+ * the same packet as cp_pack_lse, but its LSE region is a copy of a
+ * materialized LSE tensor (element strides sl) moved into the packet layout,
+ * instead of being formed from max/sum. cp_lse_materialize followed by this
+ * call gives the packet of cp_pack_lse bit for bit.
+ */
+CPLSE_API cp_status cp_pack_from_lse(const void* o, cp_strides3 so, const float* lse,
+                                     cp_strides3 sl, int W, int64_t T, int H, int D, cp_dtype dt,
+                                     int scatter_dim, void* pkt_o, float* pkt_lse, void* stream);
+
+/*
  * [DCP] "HCCL All2All" of the packet, emulated on one GPU: W simulated ranks
  * each hold W blocks of `block_bytes`; block j of rank r lands as block r of
  * rank j:  recv[j][r] = send[r][j]. Call it once per packet region (payload

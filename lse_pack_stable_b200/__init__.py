@@ -37,7 +37,8 @@ CP_OK, CP_ERR_ARG, CP_ERR_SHAPE, CP_ERR_ALIGN, CP_ERR_ALIAS, CP_ERR_UNSUPPORTED,
 CP_BF16, CP_FP16 = 0, 1
 STATUS_NAMES = {0: "CP_OK", -1: "CP_ERR_ARG", -2: "CP_ERR_SHAPE", -3: "CP_ERR_ALIGN",
                 -4: "CP_ERR_ALIAS", -5: "CP_ERR_UNSUPPORTED", -6: "CP_ERR_CUDA"}
-EXPORTS = ("cp_abi_version", "cp_last_error", "cp_pack_lse", "cp_a2a_local_permute",
+EXPORTS = ("cp_abi_version", "cp_last_error", "cp_pack_lse", "cp_lse_materialize",
+           "cp_pack_from_lse", "cp_a2a_local_permute",
            "cp_lse_combine", "cp_pack_permute_combine_fused", "ulysses_seq2head",
            "ulysses_head2seq")
 
@@ -53,13 +54,16 @@ _lib.cp_last_error.argtypes = []
 _lib.cp_last_error.restype = ctypes.c_char_p
 _lib.cp_pack_lse.argtypes = [_p, Strides3, _p, Strides3, _p, Strides3, _i, _i64, _i, _i, _i, _i,
                              _p, _p, _p]
+_lib.cp_lse_materialize.argtypes = [_p, Strides3, _p, Strides3, _i, _i64, _i, _p, _p]
+_lib.cp_pack_from_lse.argtypes = [_p, Strides3, _p, Strides3, _i, _i64, _i, _i, _i, _i, _p, _p, _p]
 _lib.cp_a2a_local_permute.argtypes = [_p, _p, _i, _i64, _p]
 _lib.cp_lse_combine.argtypes = [_p, _p, _i, _i64, _i, _i, _i, _p, _p, _p]
 _lib.cp_pack_permute_combine_fused.argtypes = [_p, Strides3, _p, Strides3, _p, Strides3, _i, _i64,
                                                _i, _i, _i, _p, _p, _p]
 _lib.ulysses_seq2head.argtypes = [_p, _p, _i, _i, _i64, _i, _i, _i, _p]
 _lib.ulysses_head2seq.argtypes = [_p, _p, _i, _i, _i64, _i, _i, _i, _p]
-for _f in ("cp_pack_lse", "cp_a2a_local_permute", "cp_lse_combine",
+for _f in ("cp_pack_lse", "cp_lse_materialize", "cp_pack_from_lse", "cp_a2a_local_permute",
+           "cp_lse_combine",
            "cp_pack_permute_combine_fused", "ulysses_seq2head", "ulysses_head2seq"):
     getattr(_lib, _f).restype = _i
 
@@ -129,6 +133,36 @@ def cp_pack_lse(o: torch.Tensor, smax: torch.Tensor, ssum: torch.Tensor, scatter
     _check(_lib.cp_pack_lse(_ptr(o), _strides3(o), _ptr(smax), _strides3(smax), _ptr(ssum),
                             _strides3(ssum), W, T, H, D, _dtype(o), scatter_dim, _ptr(pkt_o),
                             _ptr(pkt_lse), _stream(stream)))
+    return pkt_o, pkt_lse
+
+
+def cp_lse_materialize(smax: torch.Tensor, ssum: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    """Legacy first step: LSE [W, T, H] float32 from softmax max/sum."""
+    W, T, H = smax.shape
+    if lse is None:
+        lse = torch.empty((W, T, H), dtype=torch.float32, device=smax.device)
+    _dense(lse, "lse")
+    _check(_lib.cp_lse_materialize(_ptr(smax), _strides3(smax), _ptr(ssum), _strides3(ssum), W, T,
+                                   H, _ptr(lse), _stream(stream)))
+    return lse
+
+
+def cp_pack_from_lse(o: torch.Tensor, lse: torch.Tensor, scatter_dim: int = 1,
+                     pkt_o: Optional[torch.Tensor] = None, pkt_lse: Optional[torch.Tensor] = None,
+                     stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Legacy pack: the packet of cp_pack_lse, its LSE region copied from `lse`."""
+    W, T, H, D = o.shape
+    shape = (W, W, T, H // W) if scatter_dim == 1 else (W, W, T // W, H)
+    if pkt_o is None:
+        pkt_o = torch.empty(shape + (D,), dtype=o.dtype, device=o.device)
+    if pkt_lse is None:
+        pkt_lse = torch.empty(shape, dtype=torch.float32, device=o.device)
+    _dense(pkt_o, "pkt_o")
+    _dense(pkt_lse, "pkt_lse")
+    _check(_lib.cp_pack_from_lse(_ptr(o), _strides3(o), _ptr(lse), _strides3(lse), W, T, H, D,
+                                 _dtype(o), scatter_dim, _ptr(pkt_o), _ptr(pkt_lse),
+                                 _stream(stream)))
     return pkt_o, pkt_lse
 
 

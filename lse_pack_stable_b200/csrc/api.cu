@@ -229,6 +229,82 @@ cp_status cp_pack_lse(const void* o, cp_strides3 so, const float* smax, cp_strid
     return launched(cplse::launch_pack(a, static_cast<cudaStream_t>(stream)), "cp_pack_lse");
 }
 
+cp_status cp_lse_materialize(const float* smax, cp_strides3 sm, const float* ssum,
+                             cp_strides3 ss, int W, int64_t T, int H, float* lse, void* stream)
+{
+    TRY(check_dims(W, T, H, 8, CP_BF16));
+    if (T == 0) return ok();
+    TRY(check_null(smax, "smax"));
+    TRY(check_null(ssum, "ssum"));
+    TRY(check_null(lse, "lse"));
+    TRY(check_align(smax, 4, "smax"));
+    TRY(check_align(ssum, 4, "ssum"));
+    TRY(check_align(lse, 4, "lse"));
+    TRY(check_strides(sm, false, "smax"));
+    TRY(check_strides(ss, false, "ssum"));
+    const int64_t rows = (int64_t)W * T * H;
+    const Span in[2] = {strided_span(smax, W, T, H, 1, sm, 4, "smax"),
+                        strided_span(ssum, W, T, H, 1, ss, 4, "ssum")};
+    const Span out[1] = {dense_span(lse, rows * 4, "lse")};
+    TRY(check_no_alias(in, 2, out, 1));
+    {
+        const void* p[3] = {smax, ssum, lse};
+        const char* n[3] = {"smax", "ssum", "lse"};
+        TRY(check_devices(p, n, 3));
+    }
+    cplse::PackArgs a{};
+    a.smax = smax; a.ssum = ssum;
+    a.sm_r = sm.r; a.sm_t = sm.t; a.sm_h = sm.h;
+    a.ss_r = ss.r; a.ss_t = ss.t; a.ss_h = ss.h;
+    a.W = W; a.H = H; a.T = T; a.rows = rows;
+    return launched(cplse::launch_lse_materialize(a, lse, static_cast<cudaStream_t>(stream)),
+                    "cp_lse_materialize");
+}
+
+cp_status cp_pack_from_lse(const void* o, cp_strides3 so, const float* lse, cp_strides3 sl,
+                           int W, int64_t T, int H, int D, cp_dtype dt, int scatter_dim,
+                           void* pkt_o, float* pkt_lse, void* stream)
+{
+    TRY(check_dims(W, T, H, D, dt));
+    if (scatter_dim != 0 && scatter_dim != 1)
+        return fail(CP_ERR_ARG, "scatter_dim must be 0 (tokens) or 1 (heads), got %d", scatter_dim);
+    if (scatter_dim == 0 && T % W != 0)
+        return fail(CP_ERR_SHAPE, "token scatter needs T %% W == 0 (T = %lld, W = %d)", (long long)T, W);
+    if (T == 0) return ok();
+    TRY(check_null(o, "o"));
+    TRY(check_null(lse, "lse"));
+    TRY(check_null(pkt_o, "pkt_o"));
+    TRY(check_null(pkt_lse, "pkt_lse"));
+    TRY(check_align(o, 16, "o"));
+    TRY(check_align(lse, 4, "lse"));
+    TRY(check_align(pkt_o, 16, "pkt_o"));
+    TRY(check_align(pkt_lse, 4, "pkt_lse"));
+    TRY(check_strides(so, true, "o"));
+    TRY(check_strides(sl, false, "lse"));
+    const int64_t rows = (int64_t)W * T * H;
+    const Span in[2] = {strided_span(o, W, T, H, D, so, 2, "o"),
+                        strided_span(lse, W, T, H, 1, sl, 4, "lse")};
+    const Span out[2] = {dense_span(pkt_o, rows * D * 2, "pkt_o"),
+                         dense_span(pkt_lse, rows * 4, "pkt_lse")};
+    TRY(check_no_alias(in, 2, out, 2));
+    {
+        const void* p[4] = {o, lse, pkt_o, pkt_lse};
+        const char* n[4] = {"o", "lse", "pkt_o", "pkt_lse"};
+        TRY(check_devices(p, n, 4));
+    }
+    cplse::PackArgs a{};
+    a.o = static_cast<const uint16_t*>(o);
+    a.so_r = so.r; a.so_t = so.t; a.so_h = so.h;
+    a.lse = lse;
+    a.sm_r = sl.r; a.sm_t = sl.t; a.sm_h = sl.h;
+    a.pkt_o = static_cast<uint16_t*>(pkt_o);
+    a.pkt_lse = pkt_lse;
+    a.W = W; a.H = H; a.Hc = H / W; a.D = D; a.scatter_dim = scatter_dim;
+    a.T = T; a.Tc = T / W;
+    a.rows = rows;
+    return launched(cplse::launch_pack(a, static_cast<cudaStream_t>(stream)), "cp_pack_from_lse");
+}
+
 cp_status cp_a2a_local_permute(const void* send, void* recv, int W, int64_t block_bytes,
                                void* stream)
 {

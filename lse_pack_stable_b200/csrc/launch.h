@@ -35,9 +35,10 @@ struct CombineArgs {
 struct PackArgs {
     const uint16_t* o;
     int64_t so_r, so_t, so_h;
-    const float* smax;
+    const float* smax;        // max/sum-aware pack: statistics ...
     const float* ssum;
     int64_t sm_r, sm_t, sm_h, ss_r, ss_t, ss_h;
+    const float* lse;         // ... or (legacy) a materialized LSE tensor, strides in sm_*
     uint16_t* pkt_o;
     float* pkt_lse;
     int W, H, Hc, D, scatter_dim;
@@ -62,6 +63,7 @@ cudaError_t launch_combine(const CombineArgs& a, Dtype dt, cudaStream_t s);
 cudaError_t launch_fused_async(const CombineArgs& a, Dtype dt, cudaStream_t s);
 cudaError_t launch_combine_async(const CombineArgs& a, Dtype dt, cudaStream_t s);
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t s);
+cudaError_t launch_lse_materialize(const PackArgs& a, float* lse, cudaStream_t s);
 cudaError_t launch_permute(const void* send, void* recv, int W, int64_t block_bytes,
                            cudaStream_t s);
 cudaError_t launch_ulysses(const UlyssesArgs& a, cudaStream_t s);

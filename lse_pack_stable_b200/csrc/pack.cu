@@ -36,7 +36,7 @@ __device__ __forceinline__ void divmod_pack(int64_t x, int64_t d, int64_t& q, in
     }
 }
 
-template <int G, int VPL, int U>
+template <int G, int VPL, int U, bool FROM_LSE>
 __global__ void __launch_bounds__(kPackThreads) pack_kernel(const PackArgs a)
 {
     constexpr int RPI = 32 / G;
@@ -72,10 +72,15 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const PackArgs a)
             }
             dst_row = (r * a.W + j) * block_rows + slot;
             src_row = r * a.so_r + t * a.so_t + h * a.so_h;
-            const float m = ld_stream(a.smax + r * a.sm_r + t * a.sm_t + h * a.sm_h);
-            const float s = ld_stream(a.ssum + r * a.ss_r + t * a.ss_t + h * a.ss_h);
-            const bool ok = isfinite(m) && isfinite(s) && s > 0.f;
-            st_stream(a.pkt_lse + dst_row, ok ? m + logf(s) : -INFINITY);
+            if (FROM_LSE) {
+                // legacy: the materialized LSE moves into the packet layout
+                st_stream(a.pkt_lse + dst_row, ld_stream(a.lse + r * a.sm_r + t * a.sm_t + h * a.sm_h));
+            } else {
+                const float m = ld_stream(a.smax + r * a.sm_r + t * a.sm_t + h * a.sm_h);
+                const float s = ld_stream(a.ssum + r * a.ss_r + t * a.ss_t + h * a.ss_h);
+                const bool ok = isfinite(m) && isfinite(s) && s > 0.f;
+                st_stream(a.pkt_lse + dst_row, ok ? m + logf(s) : -INFINITY);
+            }
         }
 
         // ---------------- phase B: copy the payload rows
@@ -110,12 +115,12 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const PackArgs a)
     }
 }
 
-template <int G, int VPL>
+template <int G, int VPL, bool FROM_LSE>
 cudaError_t launch_pack_inst(const PackArgs& a, cudaStream_t s)
 {
     constexpr int U0 = VPL >= 8 ? 1 : 8 / VPL;
     constexpr int U = U0 > G ? G : U0;
-    auto kern = pack_kernel<G, VPL, U>;
+    auto kern = pack_kernel<G, VPL, U, FROM_LSE>;
     static int per_sm = 0;
     if (per_sm == 0) {
         int n = 0;
@@ -132,19 +137,55 @@ cudaError_t launch_pack_inst(const PackArgs& a, cudaStream_t s)
     return cudaGetLastError();
 }
 
+template <bool FROM_LSE>
+cudaError_t launch_pack_l(const PackArgs& a, cudaStream_t s)
+{
+    const RowShape rs = row_shape(a.D);
+    switch (rs.G * 10 + rs.VPL) {
+    case 41: return launch_pack_inst<4, 1, FROM_LSE>(a, s);
+    case 81: return launch_pack_inst<8, 1, FROM_LSE>(a, s);
+    case 161: return launch_pack_inst<16, 1, FROM_LSE>(a, s);
+    case 321: return launch_pack_inst<32, 1, FROM_LSE>(a, s);
+    case 322: return launch_pack_inst<32, 2, FROM_LSE>(a, s);
+    default: return launch_pack_inst<32, 4, FROM_LSE>(a, s);
+    }
+}
+
+// Legacy first step: lse[q] for q = (r, t, h) in row-major order, four rows per
+// thread, one pass over the grid.
+constexpr int kMatThreads = 256;
+
+__global__ void __launch_bounds__(kMatThreads) lse_materialize_kernel(const PackArgs a, float* lse)
+{
+    const int64_t TH = a.T * a.H;
+    const int64_t q0 = ((int64_t)blockIdx.x * kMatThreads + threadIdx.x) * 4;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int64_t q = q0 + k;
+        if (q >= a.rows) break;
+        int64_t r, rem, t, h;
+        divmod_pack(q, TH, r, rem);
+        divmod_pack(rem, (int64_t)a.H, t, h);
+        const float m = ld_stream(a.smax + r * a.sm_r + t * a.sm_t + h * a.sm_h);
+        const float sv = ld_stream(a.ssum + r * a.ss_r + t * a.ss_t + h * a.ss_h);
+        const bool ok = isfinite(m) && isfinite(sv) && sv > 0.f;
+        st_stream(lse + q, ok ? m + logf(sv) : -INFINITY);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t s)
 {
-    const RowShape rs = row_shape(a.D);
-    switch (rs.G * 10 + rs.VPL) {
-    case 41: return launch_pack_inst<4, 1>(a, s);
-    case 81: return launch_pack_inst<8, 1>(a, s);
-    case 161: return launch_pack_inst<16, 1>(a, s);
-    case 321: return launch_pack_inst<32, 1>(a, s);
-    case 322: return launch_pack_inst<32, 2>(a, s);
-    default: return launch_pack_inst<32, 4>(a, s);
-    }
+    return a.lse != nullptr ? launch_pack_l<true>(a, s) : launch_pack_l<false>(a, s);
+}
+
+cudaError_t launch_lse_materialize(const PackArgs& a, float* lse, cudaStream_t s)
+{
+    const int64_t blocks = (a.rows + 4 * kMatThreads - 1) / (4 * kMatThreads);
+    if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    lse_materialize_kernel<<<(unsigned)blocks, kMatThreads, 0, s>>>(a, lse);
+    return cudaGetLastError();
 }
 
 }  // namespace cplse

@@ -45,6 +45,8 @@ class Oracle:
         lib.oracle_payload_round.restype = ctypes.c_uint16
         lib.oracle_pack.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _i64, _i64, _p, _i64, _i64,
                                     _i64, ctypes.c_int, _i64, _i64, _i64, ctypes.c_int, _p, _p, _p]
+        lib.oracle_pack_from_lse.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _i64, _i64,
+                                             ctypes.c_int, _i64, _i64, _i64, ctypes.c_int, _p, _p]
         lib.oracle_permute.argtypes = [_p, _p, ctypes.c_int, _i64]
         lib.oracle_combine_f64.argtypes = [ctypes.c_int, _i64, _i64, _p, _p, _p, _p]
         lib.oracle_combine.argtypes = [_p, _p, ctypes.c_int, _i64, _i64, ctypes.c_int, _p, _p, _p]
@@ -55,7 +57,7 @@ class Oracle:
                                               _p, _p, _p]
         for f in ("oracle_seq2head", "oracle_head2seq"):
             getattr(lib, f).argtypes = [_p, _p, ctypes.c_int, _i64, _i64, _i64, _i64, _i64]
-        for f in ("oracle_pack", "oracle_permute", "oracle_combine_f64", "oracle_combine",
+        for f in ("oracle_pack", "oracle_pack_from_lse", "oracle_permute", "oracle_combine_f64", "oracle_combine",
                   "oracle_fused", "oracle_fused_gathered", "oracle_seq2head", "oracle_head2seq"):
             getattr(lib, f).restype = None
 
@@ -87,6 +89,23 @@ class Oracle:
                              *_elem_strides(mx), sm.ctypes.data, *_elem_strides(sm), W, T, H, D,
                              scatter_dim, pkt_o.ctypes.data, l32.ctypes.data, l64.ctypes.data)
         return pkt_o, l32, l64
+
+    def materialize_lse(self, mx: np.ndarray, sm: np.ndarray) -> np.ndarray:
+        """The legacy first step, element by element: float64 LSE of max/sum arrays."""
+        return np.vectorize(self.lse, otypes=[np.float64])(mx.astype(np.float64),
+                                                           sm.astype(np.float64))
+
+    def pack_from_lse(self, o: np.ndarray, lse: np.ndarray, scatter_dim: int = 1):
+        """o [W,T,H,D] u16, lse [W,T,H] f32 (any strides) -> (pkt_o, pkt_lse), legacy pack."""
+        W, T, H, D = o.shape
+        assert o.dtype == np.uint16 and o.strides[3] == 2 and lse.dtype == np.float32
+        shape = (W, W, T, H // W) if scatter_dim == 1 else (W, W, T // W, H)
+        pkt_o = np.empty(shape + (D,), dtype=np.uint16)
+        pkt_l = np.empty(shape, dtype=np.float32)
+        self.lib.oracle_pack_from_lse(o.ctypes.data, *_elem_strides(o)[:3], lse.ctypes.data,
+                                      *_elem_strides(lse), W, T, H, D, scatter_dim,
+                                      pkt_o.ctypes.data, pkt_l.ctypes.data)
+        return pkt_o, pkt_l
 
     # -- all-to-all permutation --------------------------------------------------------------
     def permute(self, send: np.ndarray, W: int) -> np.ndarray:

@@ -164,6 +164,35 @@ void oracle_pack(const uint16_t* o, int64_t so_r, int64_t so_t, int64_t so_h,
     }
 }
 
+/* [DCP] the Before pipeline's pack: LSE was materialized first as its own
+ * tensor lse [W][T][H] (element strides given); "permute / reshape" moves it
+ * into the packet's LSE region while the pack copies the payload. Same layout
+ * as oracle_pack; the LSE values are copied bit for bit. */
+void oracle_pack_from_lse(const uint16_t* o, int64_t so_r, int64_t so_t, int64_t so_h,
+                          const float* lse, int64_t sl_r, int64_t sl_t, int64_t sl_h,
+                          int W, int64_t T, int64_t H, int64_t D, int scatter_dim,
+                          uint16_t* pkt_o, float* pkt_lse)
+{
+    int64_t Hc = H / W, Tc = T / W;
+    for (int64_t t = 0; t < T; ++t)
+        for (int r = 0; r < W; ++r)
+            for (int64_t h = 0; h < H; ++h) {
+                int64_t j, slot;
+                if (scatter_dim == 1) {
+                    j = h / Hc;
+                    slot = t * Hc + (h % Hc);
+                } else {
+                    j = t / Tc;
+                    slot = (t % Tc) * H + h;
+                }
+                int64_t dst_row = ((int64_t)r * W + j) * (T * Hc) + slot;
+                const uint16_t* src = o + r * so_r + t * so_t + h * so_h;
+                for (int64_t d = 0; d < D; ++d)
+                    pkt_o[dst_row * D + d] = src[d];
+                pkt_lse[dst_row] = lse[r * sl_r + t * sl_t + h * sl_h];
+            }
+}
+
 /* ------------------------------------------------------------------------- */
 /* [DCP] the all-to-all, emulated: W simulated ranks each hold W blocks, block
  * j of rank r goes to rank j and lands in slot r. recv[j][r] = send[r][j].   */

@@ -242,6 +242,28 @@ def pin_pack_layout(orc):
         assert np.array_equal(pkt_s, pkt) and np.array_equal(l64s, l64)
 
 
+def pin_pack_from_lse(orc):
+    """Legacy pack: the LSE region is the materialized LSE moved by the same map
+    as the payload (numpy reshape/transpose), bits unchanged, strided input too."""
+    rng = np.random.default_rng(11)
+    for W, T, H, D in [(2, 3, 4, 8), (4, 4, 8, 8), (3, 6, 6, 16)]:
+        o, _, _ = _iota_inputs(W, T, H, D)
+        lse = rng.standard_normal((W, T, H)).astype(np.float32)
+        lse[0, 0, 0] = -np.inf
+        Hc = H // W
+        pkt, pl = orc.pack_from_lse(o, lse, 1)
+        assert np.array_equal(pkt, o.reshape(W, T, W, Hc, D).transpose(0, 2, 1, 3, 4))
+        assert np.array_equal(pl.view(np.uint32),
+                              lse.reshape(W, T, W, Hc).transpose(0, 2, 1, 3).view(np.uint32))
+        if T % W == 0:
+            pkt0, pl0 = orc.pack_from_lse(o, lse, 0)
+            assert np.array_equal(pl0, lse.reshape(W, W, T // W, H))
+        big = np.zeros((W, T, 2 * H), dtype=np.float32)
+        big[:, :, 1::2] = lse
+        _, pls = orc.pack_from_lse(o, big[:, :, 1::2], 1)
+        assert np.array_equal(pls, pl)
+
+
 def pin_permute(orc):
     rng = np.random.default_rng(1)
     for W, blk in [(1, 24), (2, 8), (4, 12), (5, 3)]:
@@ -314,5 +336,5 @@ def pin_fused_equals_chain(orc):
 
 
 ALL_PINS = [pin_lse_golden, pin_combine_golden, pin_bruteforce_attention, pin_combine_invariants,
-            pin_payload_formats, pin_pack_layout, pin_permute, pin_ulysses,
+            pin_payload_formats, pin_pack_layout, pin_pack_from_lse, pin_permute, pin_ulysses,
             pin_fused_equals_chain]

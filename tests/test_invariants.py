@@ -123,3 +123,19 @@ def test_ulysses_round_trip_config():
     z = cp.ulysses_head2seq(y)
     torch.cuda.synchronize()
     assert torch.equal(z.view(torch.int16), x.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode"])
+def test_legacy_pipeline_equals_max_sum_pack(name):
+    """Materialize LSE, then pack from it (the Before pipeline) gives the packet of
+    the max/sum-aware pack (the After pipeline) bit for bit."""
+    wl = synth.CONFIGS[name]
+    o, m, s = synth.full_inputs(wl)
+    do, dm, ds = dev_payload(o, wl.dtype), dev_f32(m), dev_f32(s)
+    for sd in (1, 0):
+        a_o, a_l = cp.cp_pack_lse(do, dm, ds, scatter_dim=sd)
+        lse = cp.cp_lse_materialize(dm, ds)
+        b_o, b_l = cp.cp_pack_from_lse(do, lse, scatter_dim=sd)
+        torch.cuda.synchronize()
+        assert torch.equal(_bits(a_o), _bits(b_o))
+        assert torch.equal(_bits(a_l), _bits(b_l))

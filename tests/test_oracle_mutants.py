@@ -34,6 +34,8 @@ MUTANTS = {
     "fp16_exponent": ("ex - 25", "ex - 24"),
     "round_truncates": ("double q = nearbyint(a / spacing);", "double q = floor(a / spacing);"),
     "fused_chunk_offset": ("int64_t j = h / Hc, hc = h % Hc;", "int64_t j = h % W, hc = h / W;"),
+    "legacy_lse_index": ("pkt_lse[dst_row] = lse[r * sl_r + t * sl_t + h * sl_h];",
+                         "pkt_lse[dst_row] = lse[r * sl_r + h * sl_t + t * sl_h];"),
 }
 
 

@@ -278,3 +278,42 @@ def test_outputs_stay_in_bounds(wl, inputs):
     for b, p, n in [(b1, p1, n1), (b2, p2, n2), (b3, p3, n3), (b4, p4, n4), (b5, p5, n5),
                     (b6, p6, n6), (b7, p7, n7), (b8, p8, n8), (b9, p9, n9)]:
         assert _canary_ok(b, p, n)
+
+
+# ------------------------------------------------------------------------------------ legacy
+
+@pytest.mark.parametrize("wl", [CASES[0], CASES[1], CASES[3], CASES[8], CASES[10]],
+                         ids=[IDS[0], IDS[1], IDS[3], IDS[8], IDS[10]])
+def test_lse_materialize(wl, inputs, orc):
+    """Legacy first step: the standalone LSE tensor, 2 ulp of the float64 LSE."""
+    _, m, s = inputs(wl)
+    lse = cp.cp_lse_materialize(dev_f32(m), dev_f32(s))
+    torch.cuda.synchronize()
+    check_pack_lse(lse.cpu().numpy(), orc.materialize_lse(m, s), m, s)
+
+
+def test_lse_materialize_strided(orc):
+    wl = _wl("strided_stats", 3, 17, 6, 8, p_invalid=0.1)
+    _, m, s = synth.full_inputs(wl)
+    bm = torch.zeros((3, 17, 12), dtype=torch.float32, device="cuda")
+    bm[:, :, 1::2] = dev_f32(m)
+    sv = dev_f32(s).transpose(0, 1).contiguous().transpose(0, 1)
+    lse = cp.cp_lse_materialize(bm[:, :, 1::2], sv)
+    torch.cuda.synchronize()
+    check_pack_lse(lse.cpu().numpy(), orc.materialize_lse(m, s), m, s)
+
+
+@pytest.mark.parametrize("wl", [CASES[0], CASES[2], CASES[4], CASES[6], CASES[9]],
+                         ids=[IDS[0], IDS[2], IDS[4], IDS[6], IDS[9]])
+@pytest.mark.parametrize("scatter_dim", [1, 0])
+def test_pack_from_lse(wl, scatter_dim, inputs, orc):
+    """Legacy pack: payload and the materialized LSE moved into the packet, bit-exact."""
+    if scatter_dim == 0 and wl.T % wl.W:
+        pytest.skip("token scatter needs T % W == 0")
+    o, _, _ = inputs(wl)
+    lse = synth.received_lse(wl, 0.1, wl.T * wl.H).reshape(wl.W, wl.T, wl.H)
+    pkt, pl = cp.cp_pack_from_lse(dev_payload(o, wl.dtype), dev_f32(lse), scatter_dim=scatter_dim)
+    torch.cuda.synchronize()
+    ref_o, ref_l = orc.pack_from_lse(o, lse, scatter_dim)
+    assert np.array_equal(host_bits(pkt), ref_o)
+    assert np.array_equal(pl.cpu().numpy().view(np.uint32), ref_l.view(np.uint32))
