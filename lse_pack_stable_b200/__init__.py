@@ -238,3 +238,38 @@ def ulysses_head2seq(x: torch.Tensor, out: Optional[torch.Tensor] = None,
     _check(_lib.ulysses_head2seq(_ptr(x), _ptr(out), W, B, S // W, Hc * W, D, x.element_size(),
                                  _stream(stream)))
     return out
+
+
+class _SeqToHead(torch.autograd.Function):
+    """all_to_all_4D(x, 2, 1) with its adjoint: the gradient of a layout
+    permutation is the inverse permutation of the incoming gradient."""
+
+    @staticmethod
+    def forward(ctx, x):
+        return ulysses_seq2head(x.contiguous())
+
+    @staticmethod
+    def backward(ctx, g):
+        return ulysses_head2seq(g.contiguous())
+
+
+class _HeadToSeq(torch.autograd.Function):
+    """all_to_all_4D(x, 1, 2) with its adjoint (seq -> head of the gradient)."""
+
+    @staticmethod
+    def forward(ctx, x):
+        return ulysses_head2seq(x.contiguous())
+
+    @staticmethod
+    def backward(ctx, g):
+        return ulysses_seq2head(g.contiguous())
+
+
+def ulysses_seq2head_autograd(x: torch.Tensor) -> torch.Tensor:
+    """ulysses_seq2head that autograd differentiates (backward: ulysses_head2seq)."""
+    return _SeqToHead.apply(x)
+
+
+def ulysses_head2seq_autograd(x: torch.Tensor) -> torch.Tensor:
+    """ulysses_head2seq that autograd differentiates (backward: ulysses_seq2head)."""
+    return _HeadToSeq.apply(x)

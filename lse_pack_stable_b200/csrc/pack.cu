@@ -137,9 +137,87 @@ cudaError_t launch_pack_inst(const PackArgs& a, cudaStream_t s)
     return cudaGetLastError();
 }
 
+// Head-chunk pack of rank rows that are back to back (so_h == D), one packet
+// block (r, j) per grid row: the block is T rows of Hc*D contiguous elements,
+// row t copied from source (r, t) at head j*Hc. Each thread moves U 16-byte
+// vectors (all loads in flight before the first store) and the grid covers
+// the block once, so blocks retire and start continuously. The last grid
+// columns form (or, legacy, move) the block's T*Hc LSE values.
+#ifndef CPLSE_PACK_U
+#define CPLSE_PACK_U 8
+#endif
+constexpr int kBlockThreads = 256;
+constexpr int kBlockU = CPLSE_PACK_U;
+
+template <bool FROM_LSE>
+__global__ void __launch_bounds__(kBlockThreads)
+pack_block_kernel(const PackArgs a, int64_t pay_cols)
+{
+    const int rj = blockIdx.y;
+    const int r = rj / a.W, j = rj - r * a.W;
+    const int64_t HcV = (int64_t)a.Hc * (a.D >> 3);        // vectors per packet row
+    const int64_t block_rows = a.T * a.Hc;
+    if ((int64_t)blockIdx.x < pay_cols) {
+        const int64_t nvec = a.T * HcV;
+        const uint4* src = reinterpret_cast<const uint4*>(a.o + r * a.so_r + (int64_t)j * a.Hc * a.D);
+        uint4* dst = reinterpret_cast<uint4*>(a.pkt_o) + (int64_t)rj * nvec;
+        const int64_t st8 = a.so_t >> 3;
+        const int64_t base = (int64_t)blockIdx.x * kBlockThreads * kBlockU + threadIdx.x;
+        uint4 v[kBlockU];
+#pragma unroll
+        for (int u = 0; u < kBlockU; ++u) {
+            const int64_t k = base + (int64_t)u * kBlockThreads;
+            if (k < nvec) {
+                int64_t t, off;
+                divmod_pack(k, HcV, t, off);
+                v[u] = ld_stream(src + t * st8 + off);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kBlockU; ++u) {
+            const int64_t k = base + (int64_t)u * kBlockThreads;
+            if (k < nvec) st_stream(dst + k, v[u]);
+        }
+    } else {
+        const int64_t base = ((int64_t)blockIdx.x - pay_cols) * kBlockThreads * 4 + threadIdx.x;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t k = base + (int64_t)u * kBlockThreads;
+            if (k >= block_rows) break;
+            int64_t t, hc;
+            divmod_pack(k, (int64_t)a.Hc, t, hc);
+            const int64_t h = (int64_t)j * a.Hc + hc;
+            float lv;
+            if (FROM_LSE) {
+                lv = ld_stream(a.lse + r * a.sm_r + t * a.sm_t + h * a.sm_h);
+            } else {
+                const float m = ld_stream(a.smax + r * a.sm_r + t * a.sm_t + h * a.sm_h);
+                const float sv = ld_stream(a.ssum + r * a.ss_r + t * a.ss_t + h * a.ss_h);
+                const bool ok = isfinite(m) && isfinite(sv) && sv > 0.f;
+                lv = ok ? m + logf(sv) : -INFINITY;
+            }
+            st_stream(a.pkt_lse + (int64_t)rj * block_rows + k, lv);
+        }
+    }
+}
+
+template <bool FROM_LSE>
+cudaError_t launch_pack_blocks(const PackArgs& a, cudaStream_t s)
+{
+    const int64_t HcV = (int64_t)a.Hc * (a.D >> 3);
+    const int64_t pay_cols = (a.T * HcV + kBlockThreads * kBlockU - 1) / (kBlockThreads * kBlockU);
+    const int64_t lse_cols = (a.T * a.Hc + kBlockThreads * 4 - 1) / (kBlockThreads * 4);
+    if (pay_cols + lse_cols > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    dim3 grid((unsigned)(pay_cols + lse_cols), (unsigned)(a.W * a.W));
+    pack_block_kernel<FROM_LSE><<<grid, kBlockThreads, 0, s>>>(a, pay_cols);
+    return cudaGetLastError();
+}
+
 template <bool FROM_LSE>
 cudaError_t launch_pack_l(const PackArgs& a, cudaStream_t s)
 {
+    // head chunks of back-to-back rows: chunk copies; anything else: row by row
+    if (a.scatter_dim == 1 && a.so_h == a.D) return launch_pack_blocks<FROM_LSE>(a, s);
     const RowShape rs = row_shape(a.D);
     switch (rs.G * 10 + rs.VPL) {
     case 41: return launch_pack_inst<4, 1, FROM_LSE>(a, s);
