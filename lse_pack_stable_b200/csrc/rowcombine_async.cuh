@@ -143,6 +143,12 @@ rowcombine_async_kernel(const CombineArgs a)
     const int64_t my_chunks = warp < nchunks ? (nchunks - warp + nwarps - 1) / nwarps : 0;
     const int64_t ngroups = my_chunks * STEPS;
 
+    // Programmatic dependent launch: the next kernel in the stream may be
+    // scheduled now, and this one reads nothing until the previous kernel in
+    // the stream has completed and its writes are visible.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
     // payload vector offset (rank 0) of output row q
     auto row_src = [&](int64_t q) -> int64_t {
         if (MODE == kModeFused) {
