@@ -188,11 +188,17 @@ def _oracle_fmt(wl):
 
 
 def oracle_seconds_per_token(wl, o, m, s):
+    """Per-token cost of the oracle, from a sample large enough (~0.2 s of work)
+    that thread start-up does not dominate."""
     orc, fmt = _oracle_fmt(wl)
     t_cal = min(wl.T, 16, o.shape[1])
-    t0 = time.perf_counter()
-    orc.fused(o[:, :t_cal], m[:, :t_cal], s[:, :t_cal], fmt)
-    return max(time.perf_counter() - t0, 1e-6) / t_cal
+    while True:
+        t0 = time.perf_counter()
+        orc.fused(o[:, :t_cal], m[:, :t_cal], s[:, :t_cal], fmt)
+        el = time.perf_counter() - t0
+        if el > 0.2 or t_cal >= min(wl.T, o.shape[1]):
+            return max(el, 1e-6) / t_cal
+        t_cal = min(wl.T, o.shape[1], t_cal * 4)
 
 
 def time_oracle(wl: synth.Workload, budget_s: float, o=None, m=None, s=None):
@@ -202,7 +208,7 @@ def time_oracle(wl: synth.Workload, budget_s: float, o=None, m=None, s=None):
     orc, fmt = _oracle_fmt(wl)
     per_tok = wl.fused_bytes() / wl.T
     if o is None:
-        o, m, s = sample_inputs(wl, min(wl.T, 16))
+        o, m, s = sample_inputs(wl, min(wl.T, 256))
     dt = oracle_seconds_per_token(wl, o, m, s)
     toks = int(max(1, min(wl.T, budget_s / dt)))
     if o.shape[1] < toks:
@@ -397,7 +403,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, _, sample, cores = time_oracle(wl, 12.0, o_h.numpy().view(np.uint16), m_h.numpy(),
+        gbs, _, sample, cores = time_oracle(wl, 15.0, o_h.numpy().view(np.uint16), m_h.numpy(),
                                             s_h.numpy())
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                "sample": sample}

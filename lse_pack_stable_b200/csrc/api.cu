@@ -8,9 +8,6 @@
 #include "cplse.h"
 #include "launch.h"
 
-#ifndef CPLSE_FORCE_LSU
-#define CPLSE_FORCE_LSU 0
-#endif
 
 namespace cplse {
 
@@ -365,15 +362,9 @@ cp_status cp_lse_combine(const void* recv_o, const float* recv_lse, int W, int64
     a.W = W; a.H = Hc * W; a.Hc = Hc; a.D = D;
     a.T = T; a.N = N; a.rows = (int64_t)W * N;
     a.dense_rows = 1;
-#if CPLSE_FORCE_LSU
-    return launched(cplse::launch_combine(a, static_cast<cplse::Dtype>(dt),
-                                          static_cast<cudaStream_t>(stream)),
-                    "cp_lse_combine");
-#else
     return launched(cplse::launch_combine_async(a, static_cast<cplse::Dtype>(dt),
-                                              static_cast<cudaStream_t>(stream)),
+                                                static_cast<cudaStream_t>(stream)),
                     "cp_lse_combine");
-#endif
 }
 
 cp_status cp_pack_permute_combine_fused(const void* o, cp_strides3 so, const float* smax,
@@ -413,15 +404,9 @@ cp_status cp_pack_permute_combine_fused(const void* o, cp_strides3 so, const flo
     a.W = W; a.H = H; a.Hc = H / W; a.D = D;
     a.T = T; a.N = T * (H / W); a.rows = rows;
     a.dense_rows = (so.h == D && so.t == (int64_t)H * D) ? 1 : 0;
-#if CPLSE_FORCE_LSU
-    return launched(cplse::launch_fused(a, static_cast<cplse::Dtype>(dt),
-                                        static_cast<cudaStream_t>(stream)),
-                    "cp_pack_permute_combine_fused");
-#else
     return launched(cplse::launch_fused_async(a, static_cast<cplse::Dtype>(dt),
-                                            static_cast<cudaStream_t>(stream)),
+                                              static_cast<cudaStream_t>(stream)),
                     "cp_pack_permute_combine_fused");
-#endif
 }
 
 static cp_status ulysses(const void* in, void* out, int W, int B, int64_t S_local, int H, int D,

@@ -56,10 +56,9 @@ struct UlyssesArgs {
     int mode;                 // 0: seq->head, 1: head->seq
 };
 
-// register-staged merge (rowcombine.cuh)
-cudaError_t launch_fused(const CombineArgs& a, Dtype dt, cudaStream_t s);
-cudaError_t launch_combine(const CombineArgs& a, Dtype dt, cudaStream_t s);
-// shared-memory-staged merge (rowcombine_async.cuh): same arithmetic, same bits
+// the stable merge, fused (from max/sum, in place) or on a received packet:
+// shared-memory-staged (rowcombine_async.cuh) up to 8 ranks, register-staged
+// (rowcombine.cuh) from 16; same arithmetic, same bits
 cudaError_t launch_fused_async(const CombineArgs& a, Dtype dt, cudaStream_t s);
 cudaError_t launch_combine_async(const CombineArgs& a, Dtype dt, cudaStream_t s);
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t s);

@@ -301,28 +301,4 @@ cudaError_t launch_rowcombine_inst(const CombineArgs& a, cudaStream_t s)
     return cudaGetLastError();
 }
 
-template <typename P, int MODE, int WMAX>
-cudaError_t launch_rowcombine_w(const CombineArgs& a, cudaStream_t s)
-{
-    const RowShape rs = row_shape(a.D);
-    switch (rs.G * 10 + rs.VPL) {
-    case 41: return launch_rowcombine_inst<P, MODE, WMAX, 4, 1>(a, s);
-    case 81: return launch_rowcombine_inst<P, MODE, WMAX, 8, 1>(a, s);
-    case 161: return launch_rowcombine_inst<P, MODE, WMAX, 16, 1>(a, s);
-    case 321: return launch_rowcombine_inst<P, MODE, WMAX, 32, 1>(a, s);
-    case 322: return launch_rowcombine_inst<P, MODE, WMAX, 32, 2>(a, s);
-    default: return launch_rowcombine_inst<P, MODE, WMAX, 32, 4>(a, s);
-    }
-}
-
-template <typename P, int MODE>
-cudaError_t launch_rowcombine_p(const CombineArgs& a, cudaStream_t s)
-{
-    if (a.W <= 2) return launch_rowcombine_w<P, MODE, 2>(a, s);
-    if (a.W <= 4) return launch_rowcombine_w<P, MODE, 4>(a, s);
-    if (a.W <= 8) return launch_rowcombine_w<P, MODE, 8>(a, s);
-    if (a.W <= 16) return launch_rowcombine_w<P, MODE, 16>(a, s);
-    return launch_rowcombine_w<P, MODE, 32>(a, s);
-}
-
 }  // namespace cplse
