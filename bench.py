@@ -490,19 +490,20 @@ def measure_e2e(cp, wl, o_h, m_h, s_h, sets, stream, dev, K, Wm, barrier, world,
 
 
 def _time(fn, stream, reps=20):
+    """Median device time of one call: back-to-back calls, each bracketed by
+    events on the launching stream, one synchronisation at the end."""
     import torch
-    for _ in range(3):
-        fn(0)
-    torch.cuda.synchronize()
-    ts = []
-    for i in range(reps):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
+    for i in range(3):
         fn(i)
-        b.record(stream)
-        torch.cuda.synchronize()
-        ts.append(a.elapsed_time(b))
-    return statistics.median(ts)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for i in range(reps):
+        ev[i][0].record(stream)
+        fn(i)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ev)
 
 
 def measure_breakdown(cp, wl, sets, stream, dev, peak, tdt):

@@ -163,8 +163,10 @@ rowcombine_async_kernel(const CombineArgs a)
         }
     };
 
+    const bool linear_chunks = MODE == kModeFused ? a.dense_rows != 0 : (a.N & 31) == 0;
+
     // issue cursor: group ni = chunk ci_i, step st_i, ring slot sl_i
-    int64_t ni = 0, ci_i = 0;
+    int64_t ni = 0, ci_i = 0, chunk_src = 0;
     int st_i = 0, sl_i = 0;
     auto issue_next = [&]() {
         if (ni < ngroups) {
@@ -195,8 +197,12 @@ rowcombine_async_kernel(const CombineArgs a)
                 }
             }
             const int64_t q = c * 32 + st_i * RPI + sub;
+            if (st_i == 0) chunk_src = row_src(c * 32);   // rank-0 offset of the chunk's row 0
             if (q < a.rows) {
-                const uint4* base = src16 + row_src(q) + gl;
+                // rows of a chunk are consecutive rows of one block when the block
+                // row count is a multiple of 32 (combine) or rows are dense (fused)
+                const int64_t off = linear_chunks ? chunk_src + (st_i * RPI + sub) * V : row_src(q);
+                const uint4* base = src16 + off + gl;
                 uint4* sl = ring + sl_i * Ring::kSlotVecs + lane;
 #pragma unroll
                 for (int e = 0; e < VPL; ++e) {
