@@ -553,6 +553,14 @@ def measure_breakdown(cp, wl, sets, stream, dev, peak, tdt):
     unfused_us = res["pack"]["us"] + res["permute"]["us"] + res["combine"]["us"]
     res["unfused_total_us"] = round(unfused_us, 2)
     del pk, rv, outs
+    # context for the fused share at this size: a plain device-to-device copy
+    # moving the fused kernel's byte count (half read, half written), timed the
+    # same way, its source rotating over the same sets
+    half = wl.fused_bytes() // 32 * 16
+    srcs = [s[0].reshape(-1).view(torch.uint8)[:half] for s in sets]
+    dsts = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(nb)]
+    rec("copy_same_bytes", _time(lambda i: dsts[i % nb].copy_(srcs[i % n]), stream), 2 * half)
+    del srcs, dsts
     if wl.name == "ulysses":
         S_l = T // W
         xs = [torch.empty((W, 3, S_l, H, D), dtype=tdt, device=dev).normal_() for _ in range(2)]
