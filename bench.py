@@ -221,13 +221,19 @@ def time_oracle(wl: synth.Workload, budget_s: float, o=None, m=None, s=None):
     gbs = per_tok * toks * reps / el / 1e9
     sample = ("first %d of %d tokens (all W=%d ranks, all %d heads), %d pass(es), %.1f s"
               % (toks, wl.T, wl.W, wl.H, reps, el))
-    return gbs, el / reps, sample, cpu_threads()
+    return gbs, el / reps, sample, orc.threads()
 
 
-def cpu_threads():
-    n = os.environ.get("OMP_NUM_THREADS")
-    return int(n) if n else (len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity")
-                             else os.cpu_count())
+def time_oracle_threads(wl, budget_s, threads, o, m, s):
+    """time_oracle with the oracle's parallel loops on `threads` threads (the
+    previous count is restored afterwards)."""
+    orc, _ = _oracle_fmt(wl)
+    prev = orc.threads()
+    orc.set_threads(threads)
+    try:
+        return time_oracle(wl, budget_s, o, m, s)
+    finally:
+        orc.set_threads(prev)
 
 
 def sample_inputs(wl, toks):
@@ -257,7 +263,7 @@ def run_reference(args):
         if i >= warm:
             per_step.append((per_tok * toks / sec / 1e9, sec))
     sample = "first %d of %d tokens (all W=%d ranks, all %d heads) per step" % (toks, wl.T, wl.W, wl.H)
-    cores = cpu_threads()
+    cores = orc.threads()
     value = statistics.median(g for g, _ in per_step)
     line = {
         "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
@@ -403,10 +409,13 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, _, sample, cores = time_oracle(wl, 15.0, o_h.numpy().view(np.uint16), m_h.numpy(),
-                                            s_h.numpy())
+        host = (o_h.numpy().view(np.uint16), m_h.numpy(), s_h.numpy())
+        gbs, _, sample, cores = time_oracle(wl, 15.0, *host)
+        gbs1, _, sample1, _ = time_oracle_threads(wl, 5.0, 1, *host)
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-               "sample": sample}
+               "sample": sample,
+               "single_thread": {"value": round(gbs1, 4), "unit": "GB/s", "cores": 1,
+                                 "sample": sample1}}
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,

@@ -57,9 +57,20 @@ class Oracle:
                                               _p, _p, _p]
         for f in ("oracle_seq2head", "oracle_head2seq"):
             getattr(lib, f).argtypes = [_p, _p, ctypes.c_int, _i64, _i64, _i64, _i64, _i64]
+        lib.oracle_threads.argtypes = []
+        lib.oracle_threads.restype = ctypes.c_int
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_threads.restype = ctypes.c_int
         for f in ("oracle_pack", "oracle_pack_from_lse", "oracle_permute", "oracle_combine_f64", "oracle_combine",
                   "oracle_fused", "oracle_fused_gathered", "oracle_seq2head", "oracle_head2seq"):
             getattr(lib, f).restype = None
+
+    # -- threads of the parallel loops ---------------------------------------------------------
+    def threads(self) -> int:
+        return int(self.lib.oracle_threads())
+
+    def set_threads(self, n: int) -> int:
+        return int(self.lib.oracle_set_threads(int(n)))
 
     # -- scalar helpers ----------------------------------------------------------------------
     def lse(self, m: float, s: float) -> float:

@@ -36,8 +36,32 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 enum { ORACLE_BF16 = 0, ORACLE_FP16 = 1 };
+
+/* Threads of the parallel loops below (the benchmark times the oracle on all
+ * host cores and on one). oracle_set_threads returns the count now in effect. */
+int oracle_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+int oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+    return oracle_threads();
+}
 
 /* ------------------------------------------------------------------------- */
 /* payload formats, from their bit-level definitions                          */

@@ -121,7 +121,9 @@ def test_pack_strided_inputs(orc):
 # ------------------------------------------------------------------------------------ permute
 
 @pytest.mark.parametrize("W,block_bytes", [(1, 48), (2, 16), (4, 4096), (5, 3), (8, 1000),
-                                           (3, 18), (16, 64), (32, 32)])
+                                           (3, 18), (16, 64), (32, 32),
+                                           # several grid tiles per block plus a ragged tail
+                                           (6, 3 * 32768 + 24), (32, 4104)])
 def test_permute_blocks(W, block_bytes, orc):
     rng = np.random.default_rng(W * 1000 + block_bytes)
     send = rng.integers(0, 256, size=W * W * block_bytes, dtype=np.uint8)
@@ -217,6 +219,23 @@ def test_ulysses(W, B, S_l, H, D, eb, orc):
     assert np.array_equal(view(y), orc.seq2head(x))
     assert np.array_equal(view(back), x)
     assert np.array_equal(view(w), orc.head2seq(z))
+
+
+@pytest.mark.parametrize("W,B,S_l,H,D,eb", [(2, 65537, 1, 2, 4, 2), (4, 70001, 1, 4, 3, 1),
+                                              (2, 65600, 2, 2, 8, 4)])
+def test_ulysses_many_batch_planes(W, B, S_l, H, D, eb, orc):
+    """More batch planes than one grid dimension holds (B > 65535): the
+    one-warp-per-chunk launch, both directions, against the oracle."""
+    rng = np.random.default_rng(B)
+    npdt = {1: np.uint8, 2: np.uint16, 4: np.uint32}[eb]
+    sdt = {1: np.uint8, 2: np.int16, 4: np.int32}[eb]
+    x = rng.integers(0, 2 ** (8 * eb) - 1, size=(W, B, S_l, H, D), dtype=npdt)
+    y = cp.ulysses_seq2head(torch.from_numpy(x.view(sdt)).cuda())
+    back = cp.ulysses_head2seq(y)
+    torch.cuda.synchronize()
+    view = lambda t: t.cpu().numpy().view(npdt)
+    assert np.array_equal(view(y), orc.seq2head(x))
+    assert np.array_equal(view(back), x)
 
 
 # ------------------------------------------------------------------------------------ edges
