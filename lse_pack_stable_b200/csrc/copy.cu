@@ -210,13 +210,11 @@ cudaError_t launch_ulysses_v(const UlyssesArgs& a, cudaStream_t s)
     // more batch planes than a grid layer count allows: one warp per chunk
     constexpr int UNR = 4;
     constexpr int K = 2;
-    auto kern = ulysses_kernel<V, MODE, K, UNR>;
-    static int per_sm = 0;
-    if (per_sm == 0) {
-        int n = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kCopyThreads, 0);
+    constexpr auto kern = ulysses_kernel<V, MODE, K, UNR>;
+    int per_sm = 0;
+    {
+        const cudaError_t e = resident_blocks<kern>(kCopyThreads, 0, per_sm);
         if (e != cudaSuccess) return e;
-        per_sm = n > 0 ? n : 1;
     }
     const int64_t warps_per_block = kCopyThreads / 32;
     int64_t blocks = (a.nchunks + warps_per_block - 1) / warps_per_block;

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace cplse {
 
 enum class Dtype : int { kBf16 = 0, kFp16 = 1 };
@@ -69,5 +71,34 @@ cudaError_t launch_ulysses(const UlyssesArgs& a, cudaStream_t s);
 
 // Streaming multiprocessors of the current device (cached per device).
 int sm_count();
+
+// Resident blocks per SM of kernel K at this block size and dynamic shared
+// memory, on the current device. The first call on each device opts K in to
+// that much dynamic shared memory there (a per-device function attribute).
+// Cached per device and kernel; devices beyond the cache are queried each time.
+template <auto K>
+cudaError_t resident_blocks(int threads, int smem, int& blocks)
+{
+    constexpr int kCachedDevices = 64;
+    static std::atomic<int> cache[kCachedDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const bool cached = dev >= 0 && dev < kCachedDevices;
+    if (cached) {
+        blocks = cache[dev].load(std::memory_order_relaxed);
+        if (blocks > 0) return cudaSuccess;
+    }
+    if (smem > 0) {
+        e = cudaFuncSetAttribute(K, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+    }
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, K, threads, (size_t)smem);
+    if (e != cudaSuccess) return e;
+    blocks = n > 0 ? n : 1;
+    if (cached) cache[dev].store(blocks, std::memory_order_relaxed);
+    return cudaSuccess;
+}
 
 }  // namespace cplse

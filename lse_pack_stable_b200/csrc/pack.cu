@@ -120,13 +120,11 @@ cudaError_t launch_pack_inst(const PackArgs& a, cudaStream_t s)
 {
     constexpr int U0 = VPL >= 8 ? 1 : 8 / VPL;
     constexpr int U = U0 > G ? G : U0;
-    auto kern = pack_kernel<G, VPL, U, FROM_LSE>;
-    static int per_sm = 0;
-    if (per_sm == 0) {
-        int n = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kPackThreads, 0);
+    constexpr auto kern = pack_kernel<G, VPL, U, FROM_LSE>;
+    int per_sm = 0;
+    {
+        const cudaError_t e = resident_blocks<kern>(kPackThreads, 0, per_sm);
         if (e != cudaSuccess) return e;
-        per_sm = n > 0 ? n : 1;
     }
     const int64_t nchunks = (a.rows + 31) / 32;
     int64_t blocks = (nchunks + kPackThreads / 32 - 1) / (kPackThreads / 32);

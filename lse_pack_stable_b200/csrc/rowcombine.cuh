@@ -283,13 +283,11 @@ cudaError_t launch_rowcombine_inst(const CombineArgs& a, cudaStream_t s)
 {
     constexpr int U0 = (WMAX * VPL) >= kLoadsInFlight ? 1 : kLoadsInFlight / (WMAX * VPL);
     constexpr int U = U0 > G ? G : U0;
-    auto kern = rowcombine_kernel<P, MODE, WMAX, G, VPL, U>;
-    static int per_sm = 0;
-    if (per_sm == 0) {
-        int n = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kCombineThreads, 0);
+    constexpr auto kern = rowcombine_kernel<P, MODE, WMAX, G, VPL, U>;
+    int per_sm = 0;
+    {
+        const cudaError_t e = resident_blocks<kern>(kCombineThreads, 0, per_sm);
         if (e != cudaSuccess) return e;
-        per_sm = n > 0 ? n : 1;
     }
     const int64_t nchunks = (a.rows + 31) / 32;
     const int64_t warps_per_block = kCombineThreads / 32;

@@ -25,15 +25,11 @@ cudaError_t launch_async_inst(const CombineArgs& a, cudaStream_t s)
     constexpr int NST = stages_for<WMAX, VPL>();
     using Ring = AsyncRing<WMAX, G, VPL, NST>;
     constexpr int smem = (kAsyncThreads / 32) * Ring::kWarpBytes;
-    auto kern = rowcombine_async_kernel<P, MODE, WMAX, G, VPL, NST>;
-    static int per_sm = 0;
-    if (per_sm == 0) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    constexpr auto kern = rowcombine_async_kernel<P, MODE, WMAX, G, VPL, NST>;
+    int per_sm = 0;
+    {
+        const cudaError_t e = resident_blocks<kern>(kAsyncThreads, smem, per_sm);
         if (e != cudaSuccess) return e;
-        int n = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kAsyncThreads, smem);
-        if (e != cudaSuccess) return e;
-        per_sm = n > 0 ? n : 1;
     }
     const int64_t nchunks = (a.rows + 31) / 32;
     int64_t blocks = (nchunks + kAsyncThreads / 32 - 1) / (kAsyncThreads / 32);
