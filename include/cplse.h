@@ -84,10 +84,11 @@ CPLSE_API int cp_abi_version(void);
 CPLSE_API const char* cp_last_error(void);
 
 /*
- * [DCP] "max/sum-aware DCP pack, which forms the same LSE while writing the
- * packed layout" (After pipeline), with the invalid-statistic rule of the same
- * section: a non-finite softmax_max, a non-finite softmax_sum or a
- * softmax_sum <= 0 gives LSE = -inf. LSE = max + logf(sum) in fp32.
+ * [DCP] After pipeline: the pack itself turns each row's (max, sum) into its
+ * LSE, in the same pass that moves the row's payload into the packet, so no
+ * separate LSE tensor exists. Statistics that cannot describe a softmax (max
+ * not finite, sum not finite, or sum not positive) give LSE = -inf; otherwise
+ * LSE = max + logf(sum), in fp32.
  *
  *   o      payload [W][T][H][D], element strides `so` (D contiguous; so.* >= 0
  *          and multiples of 8; base 16-byte aligned)
@@ -106,9 +107,9 @@ CPLSE_API cp_status cp_pack_lse(const void* o, cp_strides3 so, const float* smax
                       cp_dtype dt, int scatter_dim, void* pkt_o, float* pkt_lse, void* stream);
 
 /*
- * [DCP] Before pipeline, first step ("materialize LSE = softmax_max +
- * log(softmax_sum)"): the legacy path the pull request keeps for compatibility
- * and regression coverage, here the A/B baseline of the max/sum-aware pack.
+ * [DCP] Before pipeline, first step: LSE computed from max and sum into a
+ * tensor of its own. The pull request keeps this older path alongside the new
+ * pack; here it is the A/B baseline of the max/sum-aware pack.
  * Writes a standalone fp32 tensor lse [W][T][H] (contiguous) with the same
  * values cp_pack_lse forms (max + logf(sum), -inf for invalid statistics).
  *   smax, ssum fp32 [W][T][H], element strides sm / ss (>= 0).
@@ -118,8 +119,8 @@ CPLSE_API cp_status cp_lse_materialize(const float* smax, cp_strides3 sm, const 
                                        void* stream);
 
 /*
- * [DCP] Before pipeline, remaining steps ("permute / reshape", "DCP pack"):
- * the same packet as cp_pack_lse, but its LSE region is a copy of a
+ * [DCP] Before pipeline, remaining steps (rearranging into packet order, then
+ * packing): the same packet as cp_pack_lse, but its LSE region is a copy of a
  * materialized LSE tensor (element strides sl) moved into the packet layout,
  * instead of being formed from max/sum. cp_lse_materialize followed by this
  * call gives the packet of cp_pack_lse bit for bit.
@@ -129,7 +130,8 @@ CPLSE_API cp_status cp_pack_from_lse(const void* o, cp_strides3 so, const float*
                                      int scatter_dim, void* pkt_o, float* pkt_lse, void* stream);
 
 /*
- * [DCP] "HCCL All2All" of the packet, emulated on one GPU: W simulated ranks
+ * [DCP] The all-to-all of the packet (HCCL on the page's hardware), emulated
+ * on one GPU: W simulated ranks
  * each hold W blocks of `block_bytes`; block j of rank r lands as block r of
  * rank j:  recv[j][r] = send[r][j]. Call it once per packet region (payload
  * block = T*Hc*D*2 bytes, LSE block = T*Hc*4 bytes). Any block size works;

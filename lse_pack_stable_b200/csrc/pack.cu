@@ -3,8 +3,8 @@
 //
 // Source: vLLM-Ascend pull request "[Performance][Attention] Fuse local SFA LSE
 // formation into DCP pack", section "What this PR does / why we need it?"
-// (After pipeline: the pack forms the same LSE while writing the packed layout;
-// invalid-statistic rule) and "How was this patch tested?" (scatter_dim 0 and
+// (After pipeline: the LSE comes out of the pack itself, with no separate LSE
+// tensor; the rule for invalid statistics) and "How was this patch tested?" (scatter_dim 0 and
 // 1, non-contiguous output/max/sum strides).
 //
 // Work split: a warp owns chunks of 32 consecutive source rows (r, t, h) in

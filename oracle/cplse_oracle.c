@@ -18,8 +18,8 @@
  *         output slices": the all_to_all_4D(x, 2, 1) / (x, 1, 2) operand shapes
  *         [B, S/W, H, D] <-> [B, S, H/W, D] in benchmark_ulysses_a2a.py and
  *         probe_ulysses_launch.py, with byte-identical parity to the NCCL path.
- *  The combine formula itself is not printed on the pages (they call it the
- *  "existing stable combine"); the oracle uses the standard log-sum-exp merge of
+ *  The combine formula itself is not printed on the pages (the pull request
+ *  reuses a stable combine it already had); the oracle uses the standard log-sum-exp merge of
  *  partial softmax results: LSE* = logsumexp_r LSE_r, O = sum_r exp(LSE_r - LSE*) O_r,
  *  with -inf contributions weighted zero and an all-invalid row giving O = 0,
  *  LSE = -inf.
@@ -189,7 +189,7 @@ void oracle_pack(const uint16_t* o, int64_t so_r, int64_t so_t, int64_t so_h,
 }
 
 /* [DCP] the Before pipeline's pack: LSE was materialized first as its own
- * tensor lse [W][T][H] (element strides given); "permute / reshape" moves it
+ * tensor lse [W][T][H] (element strides given); a rearranging step moves it
  * into the packet's LSE region while the pack copies the payload. Same layout
  * as oracle_pack; the LSE values are copied bit for bit. */
 void oracle_pack_from_lse(const uint16_t* o, int64_t so_r, int64_t so_t, int64_t so_h,

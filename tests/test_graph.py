@@ -1,9 +1,10 @@
 """CUDA-graph capture with changed-input replay.
 
-The DCP pull request ("How was this patch tested?") checks eager execution,
-graph capture, first replay and a replay after the inputs changed in place at
-fixed addresses, so that a replay reads the new contents instead of returning
-stale captured results. The same sequence here, for the fused call and the
+The DCP pull request's test section ("How was this patch tested?") covers
+CUDA-graph capture. The check here runs the call once without a graph,
+captures it, and replays it. It then overwrites the inputs in place, at the
+same addresses, and replays again: that replay has to produce the new results,
+not the captured ones. The same sequence here, for the fused call and the
 pack -> all-to-all -> combine chain, on a side stream.
 """
 from __future__ import annotations

@@ -24,33 +24,39 @@ def _bits(t):
 
 @pytest.mark.parametrize("W,S_l,H,D", [(2, 5, 4, 8), (4, 64, 8, 128), (8, 16, 48, 128)])
 def test_training_pair_gradients(W, S_l, H, D, orc):
-    g = torch.Generator(device="cuda").manual_seed(W * S_l + H)
-    x = torch.randn((W, 3, S_l, H, D), device="cuda", dtype=torch.bfloat16, generator=g,
-                    requires_grad=True)
-    y = torch.randn((W, 1, S_l * W, H // W, D), device="cuda", dtype=torch.bfloat16, generator=g,
-                    requires_grad=True)
-    dx = torch.randn((W, 3, S_l * W, H // W, D), device="cuda", dtype=torch.bfloat16, generator=g)
-    dy = torch.randn((W, 1, S_l, H, D), device="cuda", dtype=torch.bfloat16, generator=g)
-    ox = cp.ulysses_seq2head_autograd(x)
-    oy = cp.ulysses_head2seq_autograd(y)
-    gx, gy = torch.autograd.grad((ox, oy), (x, y), (dx, dy))
+    gen = torch.Generator(device="cuda").manual_seed(W * S_l + H)
+
+    def bf16(shape, grad=False):
+        return torch.randn(shape, device="cuda", dtype=torch.bfloat16, generator=gen,
+                           requires_grad=grad)
+
+    seq_shape, head_shape = (W, 3, S_l, H, D), (W, 3, S_l * W, H // W, D)
+    qkv = bf16(seq_shape, grad=True)                                # sequence-sharded q/k/v
+    attn = bf16((W, 1, S_l * W, H // W, D), grad=True)              # head-sharded attention output
+    upstream_heads = bf16(head_shape)                               # d loss / d seq2head(qkv)
+    upstream_seq = bf16((W, 1, S_l, H, D))                          # d loss / d head2seq(attn)
+    heads = cp.ulysses_seq2head_autograd(qkv)
+    tokens = cp.ulysses_head2seq_autograd(attn)
+    grad_qkv, grad_attn = torch.autograd.grad(outputs=[heads, tokens], inputs=[qkv, attn],
+                                              grad_outputs=[upstream_heads, upstream_seq])
     torch.cuda.synchronize()
-    assert np.array_equal(_bits(ox), orc.seq2head(_bits(x)))
-    assert np.array_equal(_bits(oy), orc.head2seq(_bits(y)))
-    assert np.array_equal(_bits(gx), orc.head2seq(_bits(dx)))
-    assert np.array_equal(_bits(gy), orc.seq2head(_bits(dy)))
+    # forward: the layouts; backward: each gradient is the inverse layout of its upstream
+    assert np.array_equal(_bits(heads), orc.seq2head(_bits(qkv)))
+    assert np.array_equal(_bits(tokens), orc.head2seq(_bits(attn)))
+    assert np.array_equal(_bits(grad_qkv), orc.head2seq(_bits(upstream_heads)))
+    assert np.array_equal(_bits(grad_attn), orc.seq2head(_bits(upstream_seq)))
 
 
 def test_pair_graph_capture_and_changed_input_replay():
     W, S_l, H, D = 8, 512, 48, 128
-    x = torch.randn((W, 3, S_l, H, D), device="cuda", dtype=torch.bfloat16)
-    y = torch.randn((W, 1, S_l * W, H // W, D), device="cuda", dtype=torch.bfloat16)
-    ox = torch.empty((W, 3, S_l * W, H // W, D), device="cuda", dtype=torch.bfloat16)
-    oy = torch.empty((W, 1, S_l, H, D), device="cuda", dtype=torch.bfloat16)
+    qkv = torch.randn((W, 3, S_l, H, D), device="cuda", dtype=torch.bfloat16)
+    attn = torch.randn((W, 1, S_l * W, H // W, D), device="cuda", dtype=torch.bfloat16)
+    heads = torch.empty((W, 3, S_l * W, H // W, D), device="cuda", dtype=torch.bfloat16)
+    tokens = torch.empty((W, 1, S_l, H, D), device="cuda", dtype=torch.bfloat16)
 
     def pair(stream=None):
-        cp.ulysses_seq2head(x, out=ox, stream=stream)
-        cp.ulysses_head2seq(y, out=oy, stream=stream)
+        cp.ulysses_seq2head(qkv, out=heads, stream=stream)
+        cp.ulysses_head2seq(attn, out=tokens, stream=stream)
 
     pair()
     torch.cuda.synchronize()
@@ -60,14 +66,14 @@ def test_pair_graph_capture_and_changed_input_replay():
     with torch.cuda.graph(graph, stream=side):
         pair(stream=side)
     torch.cuda.current_stream().wait_stream(side)
-    x.normal_()
-    y.normal_()
+    qkv.normal_()                       # new contents at the captured addresses
+    attn.normal_()
     graph.replay()
     torch.cuda.synchronize()
-    got = (ox.clone(), oy.clone())
-    pair()
+    replayed = (heads.clone(), tokens.clone())
+    pair()                              # eager on the same new inputs
     torch.cuda.synchronize()
-    assert torch.equal(got[0].view(torch.int16), ox.view(torch.int16))
-    assert torch.equal(got[1].view(torch.int16), oy.view(torch.int16))
-    assert torch.equal(cp.ulysses_head2seq(ox).view(torch.int16), x.view(torch.int16))
+    assert torch.equal(replayed[0].view(torch.int16), heads.view(torch.int16))
+    assert torch.equal(replayed[1].view(torch.int16), tokens.view(torch.int16))
+    assert torch.equal(cp.ulysses_head2seq(heads).view(torch.int16), qkv.view(torch.int16))
     del graph
