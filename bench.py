@@ -337,7 +337,7 @@ def run_ours(args):
     # pre-marshalled C-ABI arguments: the timed loop is one ctypes call per step
     def cargs(oi, mi, si, out, ol):
         return (oi.data_ptr(), cp._strides3(oi), mi.data_ptr(), cp._strides3(mi), si.data_ptr(),
-                cp._strides3(si), W, T, H, D, cp._dtype(oi), out.data_ptr(), ol.data_ptr(), sh)
+                cp._strides3(si), W, T, H, D, cp._dtype(oi), 1, out.data_ptr(), ol.data_ptr(), sh)
     call_args = [cargs(*st) for st in sets]
     fused = cp._lib.cp_pack_permute_combine_fused
 

@@ -55,7 +55,7 @@ extern "C" {
 #define CPLSE_API
 #endif
 
-#define CPLSE_ABI_VERSION 1
+#define CPLSE_ABI_VERSION 2
 #define CPLSE_MAX_W 32     /* simulated ranks per call */
 #define CPLSE_MAX_D 1024   /* head dim, elements */
 
@@ -156,17 +156,24 @@ CPLSE_API cp_status cp_lse_combine(const void* recv_o, const float* recv_lse, in
                          int D, cp_dtype dt, void* out, float* out_lse, void* stream);
 
 /*
- * pack (head chunks) -> a2a -> combine in one pass: output row (j, t, hc)
- * reads row (t, j*Hc + hc) of every rank's o/smax/ssum directly. Inputs as in
- * cp_pack_lse; outputs as in cp_lse_combine with N = T*Hc:
- *   out [W][T][Hc][D], out_lse [W][T][Hc].
- * Bit-identical to cp_pack_lse(scatter_dim=1) -> cp_a2a_local_permute (both
- * regions) -> cp_lse_combine.
+ * pack -> a2a -> combine in one pass: each output row reads its source row of
+ * every rank's o/smax/ssum directly, so the packet never exists. Inputs as in
+ * cp_pack_lse. Outputs are what cp_lse_combine gives on the received packet:
+ *   scatter_dim 1 (head chunks; H % W == 0): destination j holds heads
+ *            j*Hc .. j*Hc+Hc-1 of every token:
+ *            out [W][T][Hc][D], out_lse [W][T][Hc]; row (j, t, hc) reads (t, j*Hc + hc)
+ *   scatter_dim 0 (token chunks; T % W == 0, Tc = T / W): destination j holds
+ *            tokens j*Tc .. j*Tc+Tc-1 with all heads:
+ *            out [W][Tc][H][D], out_lse [W][Tc][H]; row (j, tc, h) reads (j*Tc + tc, h),
+ *            i.e. [T][H] in source order
+ * Bit-identical to cp_pack_lse(scatter_dim) -> cp_a2a_local_permute (both
+ * regions) -> cp_lse_combine (with T/W as T and H as Hc for token chunks).
+ * out: 16-byte aligned, contiguous; out_lse: 4-byte aligned, contiguous.
  */
 CPLSE_API cp_status cp_pack_permute_combine_fused(const void* o, cp_strides3 so, const float* smax,
                                         cp_strides3 sm, const float* ssum, cp_strides3 ss, int W,
-                                        int64_t T, int H, int D, cp_dtype dt, void* out,
-                                        float* out_lse, void* stream);
+                                        int64_t T, int H, int D, cp_dtype dt, int scatter_dim,
+                                        void* out, float* out_lse, void* stream);
 
 /*
  * [ULY] all_to_all_4D(x, scatter_dim=2, gather_dim=1), W ranks on one GPU:

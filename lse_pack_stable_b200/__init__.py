@@ -50,6 +50,10 @@ class Strides3(ctypes.Structure):
 _p, _i, _i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
 _lib.cp_abi_version.argtypes = []
 _lib.cp_abi_version.restype = _i
+ABI_VERSION = 2           # include/cplse.h CPLSE_ABI_VERSION this binding marshals for
+if _lib.cp_abi_version() != ABI_VERSION:
+    raise ImportError("libcplse.so has ABI version %d, this binding needs %d: rebuild it with "
+                      "`python lse_pack_stable_b200/build.py`" % (_lib.cp_abi_version(), ABI_VERSION))
 _lib.cp_last_error.argtypes = []
 _lib.cp_last_error.restype = ctypes.c_char_p
 _lib.cp_pack_lse.argtypes = [_p, Strides3, _p, Strides3, _p, Strides3, _i, _i64, _i, _i, _i, _i,
@@ -59,7 +63,7 @@ _lib.cp_pack_from_lse.argtypes = [_p, Strides3, _p, Strides3, _i, _i64, _i, _i, 
 _lib.cp_a2a_local_permute.argtypes = [_p, _p, _i, _i64, _p]
 _lib.cp_lse_combine.argtypes = [_p, _p, _i, _i64, _i, _i, _i, _p, _p, _p]
 _lib.cp_pack_permute_combine_fused.argtypes = [_p, Strides3, _p, Strides3, _p, Strides3, _i, _i64,
-                                               _i, _i, _i, _p, _p, _p]
+                                               _i, _i, _i, _i, _p, _p, _p]
 _lib.ulysses_seq2head.argtypes = [_p, _p, _i, _i, _i64, _i, _i, _i, _p]
 _lib.ulysses_head2seq.argtypes = [_p, _p, _i, _i, _i64, _i, _i, _i, _p]
 for _f in ("cp_pack_lse", "cp_lse_materialize", "cp_pack_from_lse", "cp_a2a_local_permute",
@@ -199,18 +203,22 @@ def cp_lse_combine(recv_o: torch.Tensor, recv_lse: torch.Tensor,
 
 def cp_pack_permute_combine_fused(o: torch.Tensor, smax: torch.Tensor, ssum: torch.Tensor,
                                   out: Optional[torch.Tensor] = None,
-                                  out_lse: Optional[torch.Tensor] = None,
+                                  out_lse: Optional[torch.Tensor] = None, scatter_dim: int = 1,
                                   stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Head chunks (scatter_dim=1): out [W, T, H/W, D], out_lse [W, T, H/W].
+    Token chunks (scatter_dim=0): out [W, T/W, H, D], out_lse [W, T/W, H]."""
     W, T, H, D = o.shape
+    shape = (W, T, H // W) if scatter_dim == 1 else (W, T // W, H)
     if out is None:
-        out = torch.empty((W, T, H // W, D), dtype=o.dtype, device=o.device)
+        out = torch.empty(shape + (D,), dtype=o.dtype, device=o.device)
     if out_lse is None:
-        out_lse = torch.empty((W, T, H // W), dtype=torch.float32, device=o.device)
+        out_lse = torch.empty(shape, dtype=torch.float32, device=o.device)
     _dense(out, "out")
     _dense(out_lse, "out_lse")
     _check(_lib.cp_pack_permute_combine_fused(_ptr(o), _strides3(o), _ptr(smax), _strides3(smax),
                                               _ptr(ssum), _strides3(ssum), W, T, H, D, _dtype(o),
-                                              _ptr(out), _ptr(out_lse), _stream(stream)))
+                                              scatter_dim, _ptr(out), _ptr(out_lse),
+                                              _stream(stream)))
     return out, out_lse
 
 

@@ -369,10 +369,14 @@ cp_status cp_lse_combine(const void* recv_o, const float* recv_lse, int W, int64
 
 cp_status cp_pack_permute_combine_fused(const void* o, cp_strides3 so, const float* smax,
                                         cp_strides3 sm, const float* ssum, cp_strides3 ss, int W,
-                                        int64_t T, int H, int D, cp_dtype dt, void* out,
-                                        float* out_lse, void* stream)
+                                        int64_t T, int H, int D, cp_dtype dt, int scatter_dim,
+                                        void* out, float* out_lse, void* stream)
 {
     TRY(check_dims(W, T, H, D, dt));
+    if (scatter_dim != 0 && scatter_dim != 1)
+        return fail(CP_ERR_ARG, "scatter_dim must be 0 (tokens) or 1 (heads), got %d", scatter_dim);
+    if (scatter_dim == 0 && T % W != 0)
+        return fail(CP_ERR_SHAPE, "token scatter needs T %% W == 0 (T = %lld, W = %d)", (long long)T, W);
     if (T == 0) return ok();
     TRY(check_sources(o, so, smax, sm, ssum, ss));
     TRY(check_null(out, "out"));
@@ -404,6 +408,7 @@ cp_status cp_pack_permute_combine_fused(const void* o, cp_strides3 so, const flo
     a.W = W; a.H = H; a.Hc = H / W; a.D = D;
     a.T = T; a.N = T * (H / W); a.rows = rows;
     a.dense_rows = (so.h == D && so.t == (int64_t)H * D) ? 1 : 0;
+    a.token_scatter = scatter_dim == 0 ? 1 : 0;
     return launched(cplse::launch_fused_async(a, static_cast<cplse::Dtype>(dt),
                                               static_cast<cudaStream_t>(stream)),
                     "cp_pack_permute_combine_fused");

@@ -32,6 +32,8 @@ struct CombineArgs {
     int64_t N;                // combine: rows per block
     int64_t rows;             // output rows
     int dense_rows;           // fused: rank rows back to back (so_h == D, so_t == H*D)
+    int token_scatter;        // fused: token-chunk exchange, output row (t, h) = source row (t, h);
+                              // otherwise head chunks, output row (j, t, hc) for h = j*Hc + hc
 };
 
 struct PackArgs {

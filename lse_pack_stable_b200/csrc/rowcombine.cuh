@@ -91,7 +91,7 @@ __device__ __forceinline__ void row_stats(const CombineArgs& a, int64_t q, bool 
         const int64_t j = h / a.Hc;
         const int64_t hc = h - j * a.Hc;
         src_row = t * a.so_t + h * a.so_h;
-        dst_row = (j * a.T + t) * a.Hc + hc;
+        dst_row = a.token_scatter ? q : (j * a.T + t) * a.Hc + hc;
         const float* pm = a.smax + t * a.sm_t + h * a.sm_h;
         const float* ps = a.ssum + t * a.ss_t + h * a.ss_h;
         float m[WMAX], s[WMAX];

@@ -81,24 +81,6 @@ __device__ __forceinline__ void divmod_u(int64_t x, int64_t d, int64_t& q, int64
     }
 }
 
-// Output row q -> (payload element offset of rank 0, destination row).
-template <int MODE>
-__device__ __forceinline__ void row_addr(const CombineArgs& a, int64_t q, int64_t& src, int64_t& dst)
-{
-    if (MODE == kModeFused) {
-        int64_t t, h, j, hc;
-        divmod_u(q, a.H, t, h);
-        divmod_u(h, a.Hc, j, hc);
-        src = t * a.so_t + h * a.so_h;
-        dst = (j * a.T + t) * a.Hc + hc;
-    } else {
-        int64_t j, n;
-        divmod_u(q, a.N, j, n);
-        src = (j * a.W * a.N + n) * a.D;
-        dst = q;
-    }
-}
-
 // Shared memory per warp: NST payload slots of [VPL][WMAX][32 lanes] 16-byte
 // vectors; NSTAT statistics slots of [2][WMAX][32] floats; and the chunk's row
 // table: weights [32][WS] (WS = WMAX rounded up to 4, for 16-byte reads) and
@@ -239,13 +221,13 @@ rowcombine_async_kernel(const CombineArgs a)
             const bool qv = q < a.rows;
             int64_t dst = 0;
             if (qv) {
-                if (MODE == kModeFused) {
+                if (MODE == kModeFused && !a.token_scatter) {
                     int64_t t, h, j, hc;
                     divmod_u(q, a.H, t, h);
                     divmod_u(h, a.Hc, j, hc);
                     dst = (j * a.T + t) * a.Hc + hc;
                 } else {
-                    dst = q;
+                    dst = q;                                // token chunks keep source order
                 }
             }
             const float* sl = sring + (int)(ci % Ring::kStat) * Ring::kStatSlotFloats;

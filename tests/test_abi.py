@@ -41,7 +41,7 @@ def test_only_declared_symbols_are_exported():
 
 
 def test_abi_version():
-    assert cp.abi_version() == 1
+    assert cp.abi_version() == cp.ABI_VERSION == 2
 
 
 # aligned fake addresses: host checks run before any pointer is dereferenced or queried
@@ -56,10 +56,10 @@ def _pack(W=2, T=4, H=8, D=64, dt=0, sd=1, o=A, m=2 * A, s=3 * A, po=4 * A, pl=5
     return L.cp_pack_lse(o, so, m, sm, s, ss, W, T, H, D, dt, sd, po, pl, None)
 
 
-def _fused(W=2, T=4, H=8, D=64, dt=0, o=A, m=2 * A, s=3 * A, out=4 * A, ol=5 * A, so=None):
+def _fused(W=2, T=4, H=8, D=64, dt=0, o=A, m=2 * A, s=3 * A, out=4 * A, ol=5 * A, so=None, sd=1):
     so = so or S(T * H * D, H * D, D)
     return L.cp_pack_permute_combine_fused(o, so, m, S(T * H, H, 1), s, S(T * H, H, 1), W, T, H,
-                                           D, dt, out, ol, None)
+                                           D, dt, sd, out, ol, None)
 
 
 @pytest.mark.parametrize("kw,status,msg", [
@@ -116,6 +116,9 @@ def test_empty_problem_is_ok_without_pointers():
     (dict(out=A), cp.CP_ERR_ALIAS, "out overlaps input o"),
     (dict(ol=A + 4), cp.CP_ERR_ALIAS, "out_lse overlaps input o"),
     (dict(W=64, H=64), cp.CP_ERR_UNSUPPORTED, "exceeds"),
+    (dict(sd=2), cp.CP_ERR_ARG, "scatter_dim must be"),
+    (dict(sd=0, T=5), cp.CP_ERR_SHAPE, "token scatter needs T % W == 0"),
+    (dict(sd=0, out=A + 64), cp.CP_ERR_ALIAS, "out overlaps input o"),
     # o's span follows its strides: a large token stride reaches the output
     (dict(so=S(8, 3 * A // 2 // 3, 64)), cp.CP_ERR_ALIAS, "overlaps input o"),
 ])

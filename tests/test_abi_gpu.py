@@ -16,7 +16,7 @@ L = cp._lib
 
 def _fused_raw(o_ptr, m_ptr, s_ptr, out_ptr, ol_ptr, W=2, T=4, H=8, D=64):
     return L.cp_pack_permute_combine_fused(o_ptr, S(T * H * D, H * D, D), m_ptr, S(T * H, H, 1),
-                                           s_ptr, S(T * H, H, 1), W, T, H, D, 0, out_ptr, ol_ptr,
+                                           s_ptr, S(T * H, H, 1), W, T, H, D, 0, 1, out_ptr, ol_ptr,
                                            torch.cuda.current_stream().cuda_stream)
 
 

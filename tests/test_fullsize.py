@@ -107,6 +107,34 @@ def test_fullsize_fused_and_chain(name, orc):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("name", CONFIG_NAMES)
+def test_fullsize_token_scatter(name, orc):
+    """The token-chunk exchange at full size: sampled rows against the oracle,
+    and every element against the head-chunk result it permutes."""
+    wl = synth.CONFIGS[name]
+    W, T, H, D, Hc = wl.W, wl.T, wl.H, wl.D, wl.Hc
+    Tc = T // W
+    o, m, s = device_inputs(wl)
+    tok, tok_lse = cp.cp_pack_permute_combine_fused(o, m, s, scatter_dim=0)
+    torch.cuda.synchronize()
+    t, h = sample_rows(wl, seed=1)
+    ti, hi = (torch.from_numpy(x).cuda() for x in (t, h))
+    got = host_bits(tok[ti // Tc, ti % Tc, hi])
+    got_lse = tok_lse[ti // Tc, ti % Tc, hi].cpu().numpy()
+    _, rm, rs, ref, ref_lse, ref_r = oracle_rows(wl, t, h, orc)
+    check_combined(got, got_lse, ref, ref_lse, ref_r, wl.dtype, W,
+                   extra_lse_tol=lse_member_tol(rm, rs))
+    head, head_lse = cp.cp_pack_permute_combine_fused(o, m, s, scatter_dim=1)
+    torch.cuda.synchronize()
+    del o, m, s
+    assert torch.equal(head.view(torch.int16).transpose(0, 1).reshape(T, H, D),
+                       tok.view(torch.int16).reshape(T, H, D)), "token != permuted head result"
+    assert torch.equal(head_lse.view(torch.int32).transpose(0, 1).reshape(T, H),
+                       tok_lse.view(torch.int32).reshape(T, H))
+    del head, head_lse, tok, tok_lse
+    torch.cuda.empty_cache()
+
+
 def test_fullsize_ulysses(orc):
     wl = synth.CONFIGS["ulysses"]
     W, S_l = wl.W, wl.T // wl.W

@@ -59,6 +59,23 @@ def test_fused_equals_chain_shapes(W, T, H, D, dtype):
     assert torch.equal(_bits(fl), _bits(cl))
 
 
+@pytest.mark.parametrize("W,T,H,D,dtype", [(4, 4096, 32, 128, "bf16"), (3, 33, 9, 40, "fp16"),
+                                           (16, 32, 32, 128, "fp16"), (8, 16, 16, 512, "bf16")])
+def test_token_scatter_is_a_permutation_of_head_scatter(W, T, H, D, dtype):
+    """Both exchanges merge the same W contributions of each (t, h) in the same
+    order; only where the row lands differs. Head chunks put (t, j*Hc + hc) at
+    [j][t][hc], token chunks put (t, h) at [t // Tc][t % Tc][h]."""
+    wl = synth.Workload("perm", W=W, T=T, H=H, D=D, dtype=dtype, seed=T + D, p_invalid=0.05,
+                        max_sigma=9.0, sum_dist=(synth.LOGUNIFORM, 1e-3, 1e6))
+    o, m, s = synth.full_inputs(wl)
+    do, dm, ds = dev_payload(o, dtype), dev_f32(m), dev_f32(s)
+    ho, hl = cp.cp_pack_permute_combine_fused(do, dm, ds, scatter_dim=1)
+    to, tl = cp.cp_pack_permute_combine_fused(do, dm, ds, scatter_dim=0)
+    torch.cuda.synchronize()
+    assert torch.equal(_bits(ho).transpose(0, 1).reshape(T, H, D), _bits(to).reshape(T, H, D))
+    assert torch.equal(_bits(hl).transpose(0, 1).reshape(T, H), _bits(tl).reshape(T, H))
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
 def test_w1_identity(dtype):
     wl = synth.Workload("w1", W=1, T=300, H=5, D=136, dtype=dtype, seed=3, p_invalid=0.0,

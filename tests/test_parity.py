@@ -194,6 +194,69 @@ def test_fused(wl, inputs, orc):
                    extra_lse_tol=extra)
 
 
+# Token-chunk exchange: destination j combines tokens j*T/W .. of every rank,
+# all heads; the output is [T][H] in source order. T is a multiple of W here.
+TOKEN_CASES = [
+    synth.CONFIGS["tiny"],
+    _wl("tok_w3_d24", 3, 36, 6, 24),
+    _wl("tok_w5_d72_fp16", 5, 10, 10, 72, dtype="fp16"),
+    _wl("tok_w32_max", 32, 64, 32, 64),
+    _wl("tok_d1024", 2, 6, 4, 1024),
+    _wl("tok_d8", 4, 12, 4, 8),
+    _wl("tok_w1", 1, 13, 3, 16),
+    _wl("tok_w16_stress_like", 16, 48, 32, 128, dtype="fp16", o_sigma=2.0, max_sigma=10.0,
+        sum_dist=(synth.LOGUNIFORM, 1e-3, 1e6), p_invalid=0.0, p_max_inf=0.05, p_sum_zero=0.05),
+    _wl("tok_w8_mla_like", 8, 24, 16, 512, o_sigma=0.5, max_sigma=8.0,
+        sum_dist=(synth.LOGUNIFORM, 1.0, 1e5), p_invalid=0.01, p_token_invalid=0.1,
+        last_token_invalid=True),
+    _wl("tok_w7_d40", 7, 21, 14, 40, dtype="fp16", p_invalid=0.2),
+    _wl("tok_w4_d256_many_invalid", 4, 36, 8, 256, p_invalid=0.6),
+]
+
+
+@pytest.mark.parametrize("wl", TOKEN_CASES, ids=[c.name for c in TOKEN_CASES])
+def test_fused_token_scatter(wl, inputs, orc):
+    o, m, s = inputs(wl)
+    W, T, H, D = wl.W, wl.T, wl.H, wl.D
+    do, dm, ds = _dev_inputs(wl, o, m, s)
+    out, out_lse = cp.cp_pack_permute_combine_fused(do, dm, ds, scatter_dim=0)
+    assert out.shape == (W, T // W, H, D) and out_lse.shape == (W, T // W, H)
+    # the unfused token-chunk chain, bit for bit
+    pkt, pl = cp.cp_pack_lse(do, dm, ds, scatter_dim=0)
+    co, cl = cp.cp_lse_combine(cp.cp_a2a_local_permute(pkt, W), cp.cp_a2a_local_permute(pl, W))
+    torch.cuda.synchronize()
+    assert torch.equal(co.view(torch.int16), out.view(torch.int16))
+    assert torch.equal(cl.view(torch.int32), out_lse.view(torch.int32))
+    # against the oracle's direct merge of every (t, h), in source order
+    ref, ref_lse, ref_r = orc.fused_gathered(o.reshape(W, T * H, D), m.reshape(W, T * H),
+                                             s.reshape(W, T * H), FMT[wl.dtype])
+    check_combined(host_bits(out).reshape(T * H, D), out_lse.cpu().numpy().reshape(-1), ref,
+                   ref_lse, ref_r, wl.dtype, W,
+                   extra_lse_tol=lse_member_tol(m.reshape(W, -1), s.reshape(W, -1)))
+
+
+def test_fused_token_scatter_strided_inputs(orc):
+    wl = _wl("tok_strided", 4, 24, 8, 64, p_invalid=0.05)
+    o, m, s = synth.full_inputs(wl)
+    W, T, H, D = o.shape
+    big = torch.zeros((W + 1, T + 3, H + 2, D + 16), dtype=torch.bfloat16, device="cuda")
+    ov = big[1:, 2:T + 2, 1:H + 1, 8:D + 8]
+    ov.copy_(dev_payload(o, "bf16"))
+    bm = torch.zeros((W, T, 3 * H), dtype=torch.float32, device="cuda")
+    mv = bm[:, :, 1::3]
+    mv.copy_(dev_f32(m))
+    sv = dev_f32(s).transpose(0, 1).contiguous().transpose(0, 1)
+    fo, fl = cp.cp_pack_permute_combine_fused(ov, mv, sv, scatter_dim=0)
+    co, cl = cp.cp_pack_permute_combine_fused(*_dev_inputs(wl, o, m, s), scatter_dim=0)
+    torch.cuda.synchronize()
+    assert torch.equal(co.view(torch.int16), fo.view(torch.int16))
+    assert torch.equal(cl.view(torch.int32), fl.view(torch.int32))
+    ref, ref_lse, ref_r = orc.fused_gathered(o.reshape(W, T * H, D), m.reshape(W, T * H),
+                                             s.reshape(W, T * H), FMT["bf16"])
+    check_combined(host_bits(fo).reshape(T * H, D), fl.cpu().numpy().reshape(-1), ref, ref_lse,
+                   ref_r, "bf16", W, extra_lse_tol=lse_member_tol(m.reshape(W, -1), s.reshape(W, -1)))
+
+
 # ------------------------------------------------------------------------------------ Ulysses
 
 ULY = [(2, 3, 4, 4, 8, 2), (4, 1, 3, 8, 128, 2), (3, 2, 5, 6, 24, 2), (8, 3, 16, 48, 128, 2),
