@@ -47,6 +47,38 @@ CASES = [
 ]
 IDS = [c.name for c in CASES]
 
+# Token-chunk exchange: destination j combines tokens j*T/W .. of every rank,
+# all heads; the output is [T][H] in source order. T is a multiple of W here.
+TOKEN_CASES = [
+    synth.CONFIGS["tiny"],
+    _wl("tok_w3_d24", 3, 36, 6, 24),
+    _wl("tok_w5_d72_fp16", 5, 10, 10, 72, dtype="fp16"),
+    _wl("tok_w32_max", 32, 64, 32, 64),
+    _wl("tok_d1024", 2, 6, 4, 1024),
+    _wl("tok_d8", 4, 12, 4, 8),
+    _wl("tok_w1", 1, 13, 3, 16),
+    _wl("tok_w16_stress_like", 16, 48, 32, 128, dtype="fp16", o_sigma=2.0, max_sigma=10.0,
+        sum_dist=(synth.LOGUNIFORM, 1e-3, 1e6), p_invalid=0.0, p_max_inf=0.05, p_sum_zero=0.05),
+    _wl("tok_w8_mla_like", 8, 24, 16, 512, o_sigma=0.5, max_sigma=8.0,
+        sum_dist=(synth.LOGUNIFORM, 1.0, 1e5), p_invalid=0.01, p_token_invalid=0.1,
+        last_token_invalid=True),
+    _wl("tok_w7_d40", 7, 21, 14, 40, dtype="fp16", p_invalid=0.2),
+    _wl("tok_w4_d256_many_invalid", 4, 36, 8, 256, p_invalid=0.6),
+]
+
+
+def _scatter_params(cases, token_cases=TOKEN_CASES):
+    """(workload, scatter_dim) pairs: head chunks for `cases`, token chunks for
+    those of them with T % W == 0 and for `token_cases`."""
+    seen, out = set(), []
+    for sd in (1, 0):
+        for wl in cases + (token_cases if sd == 0 else []):
+            if (sd == 0 and wl.T % wl.W) or (wl.name, sd) in seen:
+                continue
+            seen.add((wl.name, sd))
+            out.append(pytest.param(wl, sd, id="%s-sd%d" % (wl.name, sd)))
+    return out
+
 
 @pytest.fixture(scope="module")
 def inputs():
@@ -72,11 +104,8 @@ def _packet_layout(a, W, T, H, scatter_dim):
 
 # ------------------------------------------------------------------------------------ pack
 
-@pytest.mark.parametrize("wl", CASES, ids=IDS)
-@pytest.mark.parametrize("scatter_dim", [1, 0])
+@pytest.mark.parametrize("wl,scatter_dim", _scatter_params(CASES))
 def test_pack(wl, scatter_dim, inputs, orc):
-    if scatter_dim == 0 and wl.T % wl.W:
-        pytest.skip("token scatter needs T % W == 0")
     o, m, s = inputs(wl)
     do, dm, ds = _dev_inputs(wl, o, m, s)
     pkt, pl = cp.cp_pack_lse(do, dm, ds, scatter_dim=scatter_dim)
@@ -192,26 +221,6 @@ def test_fused(wl, inputs, orc):
     extra = lse_member_tol(m.reshape(W, -1), s.reshape(W, -1)).reshape(T, W, H // W).transpose(1, 0, 2)
     check_combined(host_bits(out), out_lse.cpu().numpy(), ref, ref_lse, ref_r, wl.dtype, W,
                    extra_lse_tol=extra)
-
-
-# Token-chunk exchange: destination j combines tokens j*T/W .. of every rank,
-# all heads; the output is [T][H] in source order. T is a multiple of W here.
-TOKEN_CASES = [
-    synth.CONFIGS["tiny"],
-    _wl("tok_w3_d24", 3, 36, 6, 24),
-    _wl("tok_w5_d72_fp16", 5, 10, 10, 72, dtype="fp16"),
-    _wl("tok_w32_max", 32, 64, 32, 64),
-    _wl("tok_d1024", 2, 6, 4, 1024),
-    _wl("tok_d8", 4, 12, 4, 8),
-    _wl("tok_w1", 1, 13, 3, 16),
-    _wl("tok_w16_stress_like", 16, 48, 32, 128, dtype="fp16", o_sigma=2.0, max_sigma=10.0,
-        sum_dist=(synth.LOGUNIFORM, 1e-3, 1e6), p_invalid=0.0, p_max_inf=0.05, p_sum_zero=0.05),
-    _wl("tok_w8_mla_like", 8, 24, 16, 512, o_sigma=0.5, max_sigma=8.0,
-        sum_dist=(synth.LOGUNIFORM, 1.0, 1e5), p_invalid=0.01, p_token_invalid=0.1,
-        last_token_invalid=True),
-    _wl("tok_w7_d40", 7, 21, 14, 40, dtype="fp16", p_invalid=0.2),
-    _wl("tok_w4_d256_many_invalid", 4, 36, 8, 256, p_invalid=0.6),
-]
 
 
 @pytest.mark.parametrize("wl", TOKEN_CASES, ids=[c.name for c in TOKEN_CASES])
@@ -385,13 +394,11 @@ def test_lse_materialize_strided(orc):
     check_pack_lse(lse.cpu().numpy(), orc.materialize_lse(m, s), m, s)
 
 
-@pytest.mark.parametrize("wl", [CASES[0], CASES[2], CASES[4], CASES[6], CASES[9]],
-                         ids=[IDS[0], IDS[2], IDS[4], IDS[6], IDS[9]])
-@pytest.mark.parametrize("scatter_dim", [1, 0])
+@pytest.mark.parametrize("wl,scatter_dim", _scatter_params(
+    [CASES[0], CASES[2], CASES[4], CASES[6], CASES[9]],
+    token_cases=[TOKEN_CASES[1], TOKEN_CASES[3], TOKEN_CASES[5]]))
 def test_pack_from_lse(wl, scatter_dim, inputs, orc):
     """Legacy pack: payload and the materialized LSE moved into the packet, bit-exact."""
-    if scatter_dim == 0 and wl.T % wl.W:
-        pytest.skip("token scatter needs T % W == 0")
     o, _, _ = inputs(wl)
     lse = synth.received_lse(wl, 0.1, wl.T * wl.H).reshape(wl.W, wl.T, wl.H)
     pkt, pl = cp.cp_pack_from_lse(dev_payload(o, wl.dtype), dev_f32(lse), scatter_dim=scatter_dim)
