@@ -562,6 +562,16 @@ def measure_breakdown(cp, wl, sets, stream, dev, peak, tdt):
     unfused_us = res["pack"]["us"] + res["permute"]["us"] + res["combine"]["us"]
     res["unfused_total_us"] = round(unfused_us, 2)
     del pk, rv, outs
+    if T % W == 0:
+        # the fused exchange of token chunks (same bytes, output in source order)
+        touts = [(torch.empty((W, T // W, H, D), dtype=tdt, device=dev),
+                  torch.empty((W, T // W, H), dtype=torch.float32, device=dev)) for _ in range(nb)]
+        rec("fused_token_chunks",
+            _time(lambda i: cp.cp_pack_permute_combine_fused(*sets[i % n][:3], out=touts[i % nb][0],
+                                                             out_lse=touts[i % nb][1], scatter_dim=0,
+                                                             stream=stream), stream),
+            wl.fused_bytes())
+        del touts
     # context for the fused share at this size: a plain device-to-device copy
     # moving the fused kernel's byte count (half read, half written), timed the
     # same way, its source rotating over the same sets

@@ -37,9 +37,14 @@ def test_graph_capture_and_changed_input_replay():
     pl = torch.empty((W, W, T, Hc), dtype=torch.float32, device="cuda")
     ro, rl = torch.empty_like(pkt), torch.empty_like(pl)
     co, cl = torch.empty_like(out), torch.empty_like(out_lse)
+    tout = torch.empty((W, T // W, H, D), dtype=torch.bfloat16, device="cuda")
+    tlse = torch.empty((W, T // W, H), dtype=torch.float32, device="cuda")
+    results = (out, out_lse, co, cl, tout, tlse)
 
     def step(stream=None):
         cp.cp_pack_permute_combine_fused(do, dm, ds, out=out, out_lse=out_lse, stream=stream)
+        cp.cp_pack_permute_combine_fused(do, dm, ds, out=tout, out_lse=tlse, scatter_dim=0,
+                                         stream=stream)
         cp.cp_pack_lse(do, dm, ds, pkt_o=pkt, pkt_lse=pl, stream=stream)
         cp.cp_a2a_local_permute(pkt, W, recv=ro, stream=stream)
         cp.cp_a2a_local_permute(pl, W, recv=rl, stream=stream)
@@ -47,7 +52,7 @@ def test_graph_capture_and_changed_input_replay():
 
     step()
     torch.cuda.synchronize()
-    eager = [_bits(t).clone() for t in (out, out_lse, co, cl)]
+    eager = [_bits(t).clone() for t in results]
 
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -55,11 +60,11 @@ def test_graph_capture_and_changed_input_replay():
     with torch.cuda.graph(graph, stream=side):
         step(stream=side)
     torch.cuda.current_stream().wait_stream(side)
-    for t in (out, out_lse, co, cl):
+    for t in results:
         t.zero_()
     graph.replay()
     torch.cuda.synchronize()
-    for want, got in zip(eager, (out, out_lse, co, cl)):
+    for want, got in zip(eager, results):
         assert torch.equal(want, _bits(got))
 
     # change the inputs in place (same addresses), replay, compare with eager
@@ -71,11 +76,14 @@ def test_graph_capture_and_changed_input_replay():
     ds.copy_(dev_f32(s2))
     graph.replay()
     torch.cuda.synchronize()
-    replayed = [_bits(t).clone() for t in (out, out_lse, co, cl)]
+    replayed = [_bits(t).clone() for t in results]
     assert not torch.equal(replayed[0], eager[0]), "replay returned stale results"
     step()
     torch.cuda.synchronize()
-    for want, got in zip(replayed, (out, out_lse, co, cl)):
+    for want, got in zip(replayed, results):
         assert torch.equal(want, _bits(got))
     assert torch.equal(replayed[0], replayed[2]) and torch.equal(replayed[1], replayed[3])
+    # token chunks: the head-chunk rows in source order
+    assert torch.equal(replayed[0].transpose(0, 1).reshape(T, H, D), replayed[4].reshape(T, H, D))
+    assert torch.equal(replayed[1].transpose(0, 1).reshape(T, H), replayed[5].reshape(T, H))
     del graph
