@@ -28,6 +28,13 @@ def _ptr(a: Optional[np.ndarray]):
     return None if a is None else a.ctypes.data
 
 
+def _check_split(W: int, T: int, H: int, scatter_dim: int) -> None:
+    """The packet splits heads (and, for token chunks, tokens) evenly over W ranks."""
+    assert W >= 1 and H % W == 0, "H = %d must be a multiple of W = %d" % (H, W)
+    assert scatter_dim in (0, 1) and (scatter_dim == 1 or T % W == 0), \
+        "token chunks need T %% W == 0 (T = %d, W = %d)" % (T, W)
+
+
 def _elem_strides(a: np.ndarray):
     return [s // a.itemsize for s in a.strides]
 
@@ -89,6 +96,7 @@ class Oracle:
         W, T, H, D = o.shape
         assert o.dtype == np.uint16 and o.strides[3] == 2
         assert mx.dtype == np.float32 and sm.dtype == np.float32
+        _check_split(W, T, H, scatter_dim)
         if scatter_dim == 1:
             shape = (W, W, T, H // W)
         else:
@@ -110,6 +118,7 @@ class Oracle:
         """o [W,T,H,D] u16, lse [W,T,H] f32 (any strides) -> (pkt_o, pkt_lse), legacy pack."""
         W, T, H, D = o.shape
         assert o.dtype == np.uint16 and o.strides[3] == 2 and lse.dtype == np.float32
+        _check_split(W, T, H, scatter_dim)
         shape = (W, W, T, H // W) if scatter_dim == 1 else (W, W, T // W, H)
         pkt_o = np.empty(shape + (D,), dtype=np.uint16)
         pkt_l = np.empty(shape, dtype=np.float32)
@@ -160,6 +169,7 @@ class Oracle:
         """o [W,T,H,D] u16, max/sum [W,T,H] f32 -> (out [W,T,Hc,D] f64, out_lse [W,T,Hc], rounded)."""
         W, T, H, D = o.shape
         assert o.strides[3] == 2
+        _check_split(W, T, H, 1)
         out = np.empty((W, T, H // W, D))
         out_lse = np.empty((W, T, H // W))
         rounded = np.empty((W, T, H // W, D), dtype=np.uint16)

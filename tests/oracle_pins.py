@@ -335,6 +335,32 @@ def pin_fused_equals_chain(orc):
             assert np.array_equal(g_out, f_out[j, t, hc]) and np.array_equal(g_lse, f_lse[j, t, hc])
 
 
+def pin_token_chain_equals_direct(orc):
+    """The token-chunk exchange: pack(scatter_dim=0) -> all-to-all -> combine on
+    the oracle's own packet equals the direct merge of every (t, h) in source
+    order, exactly when every LSE is representable in float32 (sum = 1). This
+    fixes where each combined row of the token-chunk variant lands: destination
+    j holds tokens j*T/W .. (j+1)*T/W - 1 with all heads."""
+    rng = np.random.default_rng(9)
+    for W, T, H, D, dt in [(2, 4, 4, 8, BF16), (4, 8, 4, 16, FP16), (3, 6, 6, 8, BF16)]:
+        o = rng.integers(0, 65535, size=(W, T, H, D), dtype=np.uint16)
+        o = np.where((o & 0x7f80) == 0x7f80, o & 0x3fff, o).astype(np.uint16)
+        if dt == FP16:
+            o = np.where((o & 0x7c00) == 0x7c00, o & 0x3bff, o).astype(np.uint16)
+        mx = rng.normal(0, 4, (W, T, H)).astype(np.float32)
+        sm = np.ones((W, T, H), dtype=np.float32)
+        sm[rng.random((W, T, H)) < 0.2] = 0.0
+        sm[:, 1, 0] = 0.0                                   # one row invalid on every rank
+        pkt, l32, _ = orc.pack(o, mx, sm, 0)                # [src][dst][T/W][H]
+        c_out, c_lse, _ = orc.combine(orc.permute(pkt, W), orc.permute(l32, W), dt)
+        d_out, d_lse, _ = orc.fused_gathered(o.reshape(W, T * H, D), mx.reshape(W, T * H),
+                                             sm.reshape(W, T * H), dt)
+        assert c_out.shape == (W, T // W, H, D)
+        assert np.array_equal(c_out.reshape(T * H, D), d_out)
+        assert np.array_equal(c_lse.reshape(T * H), d_lse)
+        assert np.isneginf(c_lse.reshape(T, H)[1, 0]) and np.all(c_out.reshape(T, H, D)[1, 0] == 0)
+
+
 ALL_PINS = [pin_lse_golden, pin_combine_golden, pin_bruteforce_attention, pin_combine_invariants,
             pin_payload_formats, pin_pack_layout, pin_pack_from_lse, pin_permute, pin_ulysses,
-            pin_fused_equals_chain]
+            pin_fused_equals_chain, pin_token_chain_equals_direct]
