@@ -271,7 +271,7 @@ def run_reference(args):
         "ms_per_step": round(1e3 * statistics.median(sec for _, sec in per_step), 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded counter-based generator, the workload's shapes and distributions)",
-        "config": config_block(wl, 1), "impl": "reference",
+        "config": config_block(wl, world), "impl": "reference",
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -389,7 +389,7 @@ def run_ours(args):
     roofline = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": recorded_traffic(args.config),
                 "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                else "fallback 6.65 TB/s", "kernel": ("rowcombine_kernel (register-staged, fused mode)" if W >= 16
+                else "fallback 6.65 TB/s", "kernel": ("rowcombine_kernel (register-staged, fused mode)" if W > 8
                            else "rowcombine_async_kernel (shared-memory-staged, fused mode)"),
                 "algorithmic_bytes_per_launch": bytes_per_call,
                 "us_per_launch": round(mean_launch_ms * 1e3, 3),
