@@ -8,21 +8,24 @@
 #include "cplse.h"
 #include "launch.h"
 
-
 namespace cplse {
 
 int sm_count()
 {
-    static int cache[64] = {0};
+    constexpr int kCachedDevices = 64;
+    static std::atomic<int> cache[kCachedDevices];
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (cache[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-        cache[dev] = n;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;   // B200; the launch reports the error
+    const bool cached = dev >= 0 && dev < kCachedDevices;
+    if (cached) {
+        const int n = cache[dev].load(std::memory_order_relaxed);
+        if (n > 0) return n;
     }
-    return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (cached) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
 }
 
 }  // namespace cplse

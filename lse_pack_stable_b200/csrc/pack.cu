@@ -4,11 +4,12 @@
 // Source: vLLM-Ascend pull request "[Performance][Attention] Fuse local SFA LSE
 // formation into DCP pack", section "What this PR does / why we need it?"
 // (After pipeline: the LSE comes out of the pack itself, with no separate LSE
-// tensor; the rule for invalid statistics) and "How was this patch tested?" (scatter_dim 0 and
-// 1, non-contiguous output/max/sum strides).
+// tensor; the rule for invalid statistics) and "How was this patch tested?"
+// (scatter_dim 0 and 1, non-contiguous output/max/sum strides).
 //
-// Work split: a warp owns chunks of 32 consecutive source rows (r, t, h) in
-// input order. Phase A: lane i forms the LSE of row i (coalesced max/sum
+// Two kernels. Head chunks with back-to-back rows take the 2-D block copy
+// further down. Everything else takes the row kernel: a warp owns chunks of 32
+// consecutive source rows (r, t, h) in input order. Phase A: lane i forms the LSE of row i (coalesced max/sum
 // loads) and writes it to the LSE region. Phase B: G lanes copy one row's D
 // elements with 16-byte vectors; U steps of loads are in flight before the
 // first store.
