@@ -16,7 +16,7 @@ import pytest
 import torch
 
 import synth
-from gpu_util import (FMT, TORCH_DT, check_combined, check_pack_lse, dev_f32, host_bits,
+from gpu_util import (FMT, TORCH_DT, check_combined, check_pack_lse, host_bits,
                       lse_member_tol)
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
