@@ -26,6 +26,9 @@ MUTANTS = {
                            "if (lse[r] < M || M == -INFINITY)\n                M = lse[r];"),
     "pack_chunk_index": ("j = h / Hc;", "j = h % W;"),
     "pack_slot_transposed": ("slot = t * Hc + (h % Hc);", "slot = (h % Hc) * T + t;"),
+    "pack_token_chunks_interleaved": ("j = t / Tc;\n                    slot = (t % Tc) * H + h;",
+                                      "j = t % W;\n                    slot = (t / W) * H + h;"),
+    "pack_token_slot_transposed": ("slot = (t % Tc) * H + h;", "slot = h * Tc + (t % Tc);"),
     "permute_identity": ("memcpy(recv + ((int64_t)j * W + r) * block_bytes",
                          "memcpy(recv + ((int64_t)r * W + j) * block_bytes"),
     "seq2head_interleaved": ("* S + (int64_t)r * S_l + s) * Hc + hc;",
