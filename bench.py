@@ -1,15 +1,22 @@
 """Benchmark of the DCP exchange hot path on B200: fused pack -> all-to-all ->
 stable log-sum-exp combine, through the C-ABI of libcplse.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config stress]
+                    [--per-config decode,mla,ulysses] [--impl ours|reference]
 
 One step = one call of cp_pack_permute_combine_fused over one batch: the whole
 DCP path (LSE formation, head-chunk pack, the W x W block exchange, combine)
 in one pass. `value` is the effective HBM throughput of that step, algorithmic
-bytes W*T*H*(2D+8) + T*H*(2D+4) per call over the device time, summed over
-ranks (each rank runs its own independent batch: weak scaling, no collective
-on the data path). The breakdown times the unfused kernels and, for the
-Ulysses workload, the layout transforms, outside the timed region.
+bytes W*T*H*(2D+8) + T*H*(2D+4) per call over the device time of K
+back-to-back steps, summed over ranks (each rank runs its own independent
+batch: weak scaling, no collective on the data path).
+
+The headline workload is the largest single-GPU one (stress, 18.8 GB per
+call). The other large workloads (decode, mla, ulysses) are measured in the
+same run and reported under `per_config`, each with its own roofline, CPU
+baseline and kernel breakdown. The roofline of each comes from a dedicated
+pass of separately event-bracketed launches (median, p10, p90), independent
+of --steps.
 
 --impl reference times the float64 CPU oracle (rank 0 only) on a bounded
 sample of the same workload, on the host cores.
@@ -20,6 +27,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import gc
 import hashlib
 import json
 import math
@@ -40,22 +48,30 @@ import synth  # noqa: E402
 
 METRIC = "pack+permute+combine µs/call and effective HBM GB/s (% of B200 peak)"
 FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 128 << 20          # at least the B200's L2 (126 MB); fixes the rotation policy
+ROOFLINE_LAUNCHES = 50
 KERNEL_SOURCES = ["lse_pack_stable_b200/csrc/rowcombine_async.cuh",
                   "lse_pack_stable_b200/csrc/rowcombine_async.cu",
                   "lse_pack_stable_b200/csrc/rowcombine.cuh", "lse_pack_stable_b200/csrc/common.cuh"]
+PER_CONFIG_DEFAULT = "decode,mla,ulysses"
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", default="decode", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="stress", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--per-config", default=PER_CONFIG_DEFAULT,
+                    help="comma-separated workloads measured after the headline one "
+                         "(one GPU only); 'none' for the headline alone")
+    ap.add_argument("--launches", type=int, default=ROOFLINE_LAUNCHES,
+                    help="event-bracketed launches of the roofline pass (at least 50)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-breakdown", action="store_true")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def env_rank():
@@ -63,15 +79,33 @@ def env_rank():
             int(os.environ.get("WORLD_SIZE", 1)))
 
 
-def config_block(wl: synth.Workload, world: int, extra=None):
-    c = {"workload": "%s: W=%d simulated ranks, T=%d, H=%d, D=%d, %s payload, fp32 max/sum"
-                     % (wl.name, wl.W, wl.T, wl.H, wl.D, wl.dtype),
-         "W": wl.W, "T": wl.T, "H": wl.H, "D": wl.D, "payload_dtype": wl.dtype,
-         "global_batch": world, "parallelism": "replicas%d" % world,
-         "bytes_per_call": wl.fused_bytes()}
-    if extra:
-        c.update(extra)
-    return c
+def rotation_sets(wl: synth.Workload) -> int:
+    """Device copies of one call's inputs and outputs that consecutive calls
+    rotate over, so that every call reads cold HBM: one when a call's bytes
+    exceed 3x the L2 already, else enough copies to cover 3x the L2."""
+    set_bytes = wl.fused_bytes()
+    if set_bytes >= 3 * L2_BYTES:
+        return 1
+    return max(2, math.ceil(3 * L2_BYTES / set_bytes) + 1)
+
+
+def l2_note(wl: synth.Workload) -> str:
+    n = rotation_sets(wl)
+    b = wl.fused_bytes()
+    if n == 1:
+        return ("one set of inputs and outputs, %.1f GB per call (> 3x the L2): every call "
+                "streams cold HBM" % (b / 1e9))
+    return ("inputs and outputs rotate over %d device sets of %.0f MB (%.0f MB in all, > 3x the L2)"
+            % (n, b / 1e6, n * b / 1e6))
+
+
+def config_block(wl: synth.Workload, world: int):
+    """The workload's description; identical in both arms of the benchmark."""
+    return {"workload": "%s: W=%d simulated ranks, T=%d, H=%d, D=%d, %s payload, fp32 max/sum"
+                        % (wl.name, wl.W, wl.T, wl.H, wl.D, wl.dtype),
+            "W": wl.W, "T": wl.T, "H": wl.H, "D": wl.D, "payload_dtype": wl.dtype,
+            "global_batch": world, "parallelism": "replicas%d" % world,
+            "bytes_per_call": wl.fused_bytes(), "l2": l2_note(wl)}
 
 
 def reduce_max(values, world, device):
@@ -100,6 +134,23 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def peak_source(kind: str) -> str:
+    return ("measured (MEASURED_PEAKS.json hbm_gbs)" if kind == "measured"
+            else "fallback 6.65 TB/s (MEASURED_PEAKS.json absent)")
+
+
+def host_cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
@@ -109,8 +160,8 @@ def kernel_source_hash():
 
 
 def recorded_traffic(config: str):
-    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
-    if it was taken on the current kernel source (else None)."""
+    """DRAM bytes per full-size launch of the fused kernel from the committed
+    ncu summary, if it was taken on the current kernel source (else None)."""
     path = os.path.join(ROOT, "profiles", "fused_%s.md" % config)
     try:
         text = open(path).read()
@@ -123,10 +174,22 @@ def recorded_traffic(config: str):
     return int(tr.group(1))
 
 
+def merge_kernel_name(W: int) -> str:
+    return ("rowcombine_kernel (register-staged, fused mode)" if W > 8
+            else "rowcombine_async_kernel (shared-memory-staged, fused mode)")
+
+
+def pct(ms, q):
+    return float(np.percentile(np.asarray(ms, dtype=np.float64), q))
+
+
 # --------------------------------------------------------------------------------------------
-# clocks during the timed region (NVML)
+# clocks during the timed regions (NVML)
 
 class ClockSampler:
+    """Samples the SM clock and the clock-event reasons in a background thread
+    while it is running; start()/stop() may be called several times and the
+    samples accumulate (the timed region and the roofline pass)."""
     REASONS = {
         "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
         "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
@@ -137,6 +200,7 @@ class ClockSampler:
         self.samples, self.reasons, self.ok = [], set(), False
         self.period = period_s
         self._stop = threading.Event()
+        self.t = None
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -148,28 +212,33 @@ class ClockSampler:
             self.err = str(e)
             self.max_mhz = None
 
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for name, bit in self.REASONS.items():
+                if mask & bit and name != "gpu_idle":
+                    self.reasons.add(name)
+        except Exception:  # noqa: BLE001
+            pass
+
     def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for name, bit in self.REASONS.items():
-                    if mask & bit and name != "gpu_idle":
-                        self.reasons.add(name)
-            except Exception:  # noqa: BLE001
-                pass
+            self._sample()
             time.sleep(self.period)
 
-    def __enter__(self):
+    def start(self):
         if self.ok:
+            self._stop.clear()
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
-        return self
 
-    def __exit__(self, *exc):
-        if self.ok:
+    def stop(self):
+        if self.ok and self.t is not None:
             self._stop.set()
             self.t.join()
+            self._sample()          # at least one sample taken under load per window
+            self.t = None
 
     def summary(self):
         if not self.ok:
@@ -242,6 +311,19 @@ def sample_inputs(wl, toks):
     return o, np.stack([a for a, _ in ms]), np.stack([b for _, b in ms])
 
 
+def cpu_baseline(wl, o, m, s, budget_s, single_thread_s):
+    """The oracle on a bounded token sample: all host threads, and (if
+    single_thread_s > 0) one thread."""
+    gbs, _, sample, cores = time_oracle(wl, budget_s, o, m, s)
+    rec = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+           "sample": sample, "cpu_model": host_cpu_model()}
+    if single_thread_s > 0:
+        gbs1, _, sample1, _ = time_oracle_threads(wl, single_thread_s, 1, o, m, s)
+        rec["single_thread"] = {"value": round(gbs1, 4), "unit": "GB/s", "cores": 1,
+                                "sample": sample1}
+    return rec
+
+
 def run_reference(args):
     rank, _, world = env_rank()
     if rank != 0:
@@ -270,10 +352,11 @@ def run_reference(args):
         "steps": steps, "warmup": warm,
         "ms_per_step": round(1e3 * statistics.median(sec for _, sec in per_step), 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "payload_dtype": wl.dtype,
         "data": "synthetic (seeded counter-based generator, the workload's shapes and distributions)",
         "config": config_block(wl, world), "impl": "reference",
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
-                         "kind": "oracle", "sample": sample},
+                         "kind": "oracle", "sample": sample, "cpu_model": host_cpu_model()},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -283,6 +366,177 @@ def run_reference(args):
 
 # --------------------------------------------------------------------------------------------
 # GPU arm
+
+class Inputs:
+    """One workload's inputs: generated on the host (into pinned memory when
+    the end-to-end leg copies from there), uploaded once, plus the device sets
+    that consecutive calls rotate over."""
+
+    def __init__(self, wl, dev, pinned):
+        import torch
+        W, T, H, D, Hc = wl.W, wl.T, wl.H, wl.D, wl.Hc
+        self.tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float16
+        self.o_h = torch.empty((W, T, H, D), dtype=torch.int16, pin_memory=pinned)
+        self.m_h = torch.empty((W, T, H), dtype=torch.float32, pin_memory=pinned)
+        self.s_h = torch.empty((W, T, H), dtype=torch.float32, pin_memory=pinned)
+        tb = max(1, (256 << 20) // (H * D * 2))
+        on = self.o_h.numpy().view(np.uint16)
+        for r in range(W):
+            for t0 in range(0, T, tb):
+                t1 = min(T, t0 + tb)
+                synth.o_block(wl, r, t0, t1, out=on[r, t0:t1])
+            mr, sr = synth.stats_block(wl, r)
+            self.m_h[r].numpy()[...] = mr
+            self.s_h[r].numpy()[...] = sr
+        self.in_bytes = self.o_h.numel() * 2 + self.m_h.numel() * 4 + self.s_h.numel() * 4
+        self.nsets = rotation_sets(wl)
+        o_d = self.o_h.to(dev).view(self.tdt)
+        m_d = self.m_h.to(dev)
+        s_d = self.s_h.to(dev)
+        self.sets = []
+        for i in range(self.nsets):
+            oi = o_d if i == 0 else o_d.clone()
+            mi = m_d if i == 0 else m_d.clone()
+            si = s_d if i == 0 else s_d.clone()
+            out = torch.empty((W, T, Hc, D), dtype=self.tdt, device=dev)
+            ol = torch.empty((W, T, Hc), dtype=torch.float32, device=dev)
+            self.sets.append((oi, mi, si, out, ol))
+
+    def host(self):
+        return self.o_h.numpy().view(np.uint16), self.m_h.numpy(), self.s_h.numpy()
+
+
+def fused_stepper(cp, wl, sets, stream):
+    """step(i): one fused call on set i mod len(sets), with pre-marshalled
+    C-ABI arguments (one ctypes call per step)."""
+    sh = stream.cuda_stream
+
+    def cargs(oi, mi, si, out, ol):
+        return (oi.data_ptr(), cp._strides3(oi), mi.data_ptr(), cp._strides3(mi), si.data_ptr(),
+                cp._strides3(si), wl.W, wl.T, wl.H, wl.D, cp._dtype(oi), 1, out.data_ptr(),
+                ol.data_ptr(), sh)
+    call_args = [cargs(*st) for st in sets]
+    fused = cp._lib.cp_pack_permute_combine_fused
+    n = len(sets)
+
+    def step(i):
+        st = fused(*call_args[i % n])
+        if st != 0:
+            raise cp.CplseError(st, cp.last_error())
+    return step
+
+
+def hold_device(stream, ms):
+    """Keep the stream busy for about `ms` milliseconds (a bounded clock spin),
+    so that the host enqueues the launches that follow before the device
+    reaches them: a timed launch then never includes host-side issue time,
+    whatever the cost of marshalling and validating one call."""
+    import torch
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(int(ms * 1e-3 * 2.0e9))
+
+
+def time_back_to_back(step, stream, K, Wm, barrier):
+    """Device time (ms) of K back-to-back steps after Wm untimed ones, one event
+    pair around the whole region, barriers and synchronisations on both sides."""
+    import torch
+    for i in range(Wm):
+        step(i)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    hold_device(stream, 2.0)
+    a.record(stream)
+    for i in range(K):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    return a.elapsed_time(b)
+
+
+def time_launches(fn, stream, reps, warm=3):
+    """Device time (ms) of each of `reps` calls, each bracketed by its own event
+    pair on the launching stream; calls follow each other with no host wait,
+    one synchronisation at the end."""
+    import torch
+    for i in range(warm):
+        fn(i)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    hold_device(stream, max(2.0, 0.2 * reps))
+    for i in range(reps):
+        ev[i][0].record(stream)
+        fn(i)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def launch_stats(ms, nbytes, peak):
+    """Median / p10 / p90 of per-launch times and the median's throughput."""
+    med = statistics.median(ms)
+    gbs = nbytes / (med * 1e-3) / 1e9
+    return {"us": round(med * 1e3, 3),
+            "us_p10_p50_p90": [round(1e3 * pct(ms, q), 3) for q in (10, 50, 90)],
+            "bytes": nbytes, "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4),
+            "launches": len(ms)}
+
+
+def measure_workload(cp, wl, dev, stream, args, world, barrier, peak, peak_kind, headline):
+    """Everything the line reports for one workload: K back-to-back steps (the
+    throughput), a roofline pass of separately bracketed launches, and, as
+    asked for, the end-to-end leg, the kernel breakdown and the CPU baseline."""
+    import torch
+    rank, local_rank, _ = env_rank()
+    inp = Inputs(wl, dev, pinned=headline and not args.no_e2e)
+    step = fused_stepper(cp, wl, inp.sets, stream)
+    bytes_per_call = wl.fused_bytes()
+    K, Wm = max(1, args.steps), max(3, args.warmup)
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    total_ms = time_back_to_back(step, stream, K, Wm, barrier)
+    launch_ms = time_launches(step, stream, max(ROOFLINE_LAUNCHES, args.launches))
+    clocks.stop()
+    med_launch = statistics.median(launch_ms)
+    total_ms, med_launch = reduce_max([total_ms, med_launch], world, dev)
+    ms_per_step = total_ms / K
+    value = job_throughput(world, bytes_per_call, K, total_ms)
+
+    achieved = bytes_per_call / (med_launch * 1e-3) / 1e9
+    overlapped = bytes_per_call / (ms_per_step * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(wl.name),
+                "peak_source": peak_source(peak_kind), "kernel": merge_kernel_name(wl.W),
+                "algorithmic_bytes_per_launch": bytes_per_call,
+                "us_per_launch": round(med_launch * 1e3, 3),
+                "us_per_launch_p10_p50_p90": [round(1e3 * pct(launch_ms, q), 3)
+                                              for q in (10, 50, 90)],
+                "launches_timed": len(launch_ms),
+                "overlapped": {"us_per_call": round(ms_per_step * 1e3, 3),
+                               "GB/s": round(overlapped, 2),
+                               "frac": round(overlapped / peak, 4),
+                               "note": "K back-to-back calls, each scheduled while the previous "
+                                       "drains (programmatic dependent launch)"}}
+    res = {"value": value, "ms_per_step": ms_per_step, "K": K, "Wm": Wm, "roofline": roofline,
+           "clocks": clocks.summary(), "bytes_per_call": bytes_per_call}
+
+    if headline and not args.no_e2e:
+        res["e2e"] = measure_e2e(cp, wl, inp, stream, dev, K, Wm, barrier, world)
+    if not args.no_breakdown and world == 1:
+        res["breakdown"] = measure_breakdown(cp, wl, inp.sets, stream, dev, peak)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        o, m, s = inp.host()
+        res["cpu_baseline"] = cpu_baseline(wl, o, m, s, 15.0 if headline else 8.0,
+                                           5.0 if headline else 0.0)
+    del inp, step
+    gc.collect()
+    torch.cuda.empty_cache()
+    return res
+
 
 def run_ours(args):
     import torch
@@ -296,139 +550,45 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-    wl0 = synth.CONFIGS[args.config]
-    wl = synth.Workload(**{**wl0.__dict__, "seed": wl0.seed + 1000 * rank})
-    W, T, H, D, Hc = wl.W, wl.T, wl.H, wl.D, wl.Hc
-    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float16
-
-    # ---- inputs: generated on the host block by block into pinned memory (the
-    # end-to-end leg copies from there), uploaded once; extra device copies
-    # rotate so that every step reads cold HBM
-    o_h = torch.empty((W, T, H, D), dtype=torch.int16, pin_memory=True)
-    m_h = torch.empty((W, T, H), dtype=torch.float32, pin_memory=True)
-    s_h = torch.empty((W, T, H), dtype=torch.float32, pin_memory=True)
-    tb = max(1, (256 << 20) // (H * D * 2))
-    for r in range(W):
-        for t0 in range(0, T, tb):
-            t1 = min(T, t0 + tb)
-            o_h[r, t0:t1].numpy()[...] = synth.o_block(wl, r, t0, t1).view(np.int16)
-        mr, sr = synth.stats_block(wl, r)
-        m_h[r].numpy()[...] = mr
-        s_h[r].numpy()[...] = sr
-    in_bytes = o_h.numel() * 2 + m_h.numel() * 4 + s_h.numel() * 4
-    out_bytes = T * H * D * 2 + T * H * 4
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    nsets = max(2, math.ceil(3 * l2 / (in_bytes + out_bytes)) + 1)
-    nsets = min(nsets, max(2, int(40e9 // (in_bytes + out_bytes))))
-    o_d = o_h.to(dev).view(tdt)
-    m_d = m_h.to(dev)
-    s_d = s_h.to(dev)
-    sets = []
-    for i in range(nsets):
-        oi = o_d if i == 0 else o_d.clone()
-        mi = m_d if i == 0 else m_d.clone()
-        si = s_d if i == 0 else s_d.clone()
-        out = torch.empty((W, T, Hc, D), dtype=tdt, device=dev)
-        ol = torch.empty((W, T, Hc), dtype=torch.float32, device=dev)
-        sets.append((oi, mi, si, out, ol))
-    stream = torch.cuda.current_stream(dev)
-    sh = stream.cuda_stream
-
-    # pre-marshalled C-ABI arguments: the timed loop is one ctypes call per step
-    def cargs(oi, mi, si, out, ol):
-        return (oi.data_ptr(), cp._strides3(oi), mi.data_ptr(), cp._strides3(mi), si.data_ptr(),
-                cp._strides3(si), W, T, H, D, cp._dtype(oi), 1, out.data_ptr(), ol.data_ptr(), sh)
-    call_args = [cargs(*st) for st in sets]
-    fused = cp._lib.cp_pack_permute_combine_fused
-
-    def step(i):
-        st = fused(*call_args[i % nsets])
-        if st != 0:
-            raise cp.CplseError(st, cp.last_error())
-
-    bytes_per_call = wl.fused_bytes()
-    K, Wm = max(1, args.steps), max(3, args.warmup)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    for i in range(Wm):
-        step(i)
-    torch.cuda.synchronize()
-
-    # every 8th launch is bracketed by events (its duration is the kernel's);
-    # the others run back to back, as a user's stream would
-    sample_every = 8
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(0, K, sample_every)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clocks:
-        barrier()
-        torch.cuda.synchronize()
-        t_start.record(stream)
-        for i in range(K):
-            if i % sample_every == 0:
-                ev[i // sample_every][0].record(stream)
-                step(i)
-                ev[i // sample_every][1].record(stream)
-            else:
-                step(i)
-        t_end.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-    total_ms = t_start.elapsed_time(t_end)
-    launch_ms = [a.elapsed_time(b) for a, b in ev]
-    mean_launch_ms = sum(launch_ms) / len(launch_ms)
-    total_ms, mean_launch_ms = reduce_max([total_ms, mean_launch_ms], world, dev)
-    ms_per_step = total_ms / K
-    value = job_throughput(world, bytes_per_call, K, total_ms)
-
+    wl0 = synth.CONFIGS[args.config]
+    wl = synth.Workload(**{**wl0.__dict__, "seed": wl0.seed + 1000 * rank})
+    stream = torch.cuda.current_stream(dev)
     peak, peak_kind = measured_peak()
-    achieved = bytes_per_call / (mean_launch_ms * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(args.config),
-                "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                else "fallback 6.65 TB/s", "kernel": ("rowcombine_kernel (register-staged, fused mode)" if W > 8
-                           else "rowcombine_async_kernel (shared-memory-staged, fused mode)"),
-                "algorithmic_bytes_per_launch": bytes_per_call,
-                "us_per_launch": round(mean_launch_ms * 1e3, 3),
-                "launches_timed": len(launch_ms),
-                "us_per_launch_p10_p50_p90": [round(1e3 * np.percentile(launch_ms, q), 3)
-                                              for q in (10, 50, 90)]}
 
-    # ---- end to end through the C-ABI with host buffers (pinned), N GPUs
-    e2e = None
-    if not args.no_e2e:
-        e2e = measure_e2e(cp, wl, o_h, m_h, s_h, sets, stream, dev, K, Wm, barrier, world,
-                          dist, tdt)
+    head = measure_workload(cp, wl, dev, stream, args, world, barrier, peak, peak_kind, True)
 
-    breakdown = None
-    if not args.no_breakdown:
-        breakdown = measure_breakdown(cp, wl, sets, stream, dev, peak, tdt)
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        host = (o_h.numpy().view(np.uint16), m_h.numpy(), s_h.numpy())
-        gbs, _, sample, cores = time_oracle(wl, 15.0, *host)
-        gbs1, _, sample1, _ = time_oracle_threads(wl, 5.0, 1, *host)
-        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-               "sample": sample,
-               "single_thread": {"value": round(gbs1, 4), "unit": "GB/s", "cores": 1,
-                                 "sample": sample1}}
+    per_config = None
+    names = [] if args.per_config in ("", "none") else args.per_config.split(",")
+    if world == 1 and names:
+        per_config = {}
+        for name in names:
+            if name == args.config:
+                continue
+            r = measure_workload(cp, synth.CONFIGS[name], dev, stream, args, 1, barrier, peak,
+                                 peak_kind, False)
+            per_config[name] = {
+                "config": config_block(synth.CONFIGS[name], 1),
+                "us_per_call": round(r["ms_per_step"] * 1e3, 3),
+                "GB/s": round(r["value"], 2), "steps": r["K"], "roofline": r["roofline"],
+                "clocks": r["clocks"], "cpu_baseline": r.get("cpu_baseline"),
+                "breakdown": r.get("breakdown")}
 
     line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-        "steps": K, "warmup": Wm, "ms_per_step": round(ms_per_step, 5),
-        "us_per_call": round(ms_per_step * 1e3, 3),
+        "metric": METRIC, "value": round(head["value"], 2), "unit": "GB/s", "n_gpus": world,
+        "steps": head["K"], "warmup": head["Wm"], "ms_per_step": round(head["ms_per_step"], 5),
+        "us_per_call": round(head["ms_per_step"] * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "payload_dtype": wl.dtype,
         "data": "synthetic (seeded counter-based generator, the workload's shapes and distributions)",
-        "config": config_block(wl, world, {
-            "l2": "inputs and outputs rotate over %d device sets (%.0f MB each, %.0f MB total > "
-                  "3x the %.0f MB L2)" % (nsets, (in_bytes + out_bytes) / 1e6,
-                                          nsets * (in_bytes + out_bytes) / 1e6, l2 / 1e6)}),
-        "roofline": roofline, "clocks": clocks.summary(), "gpu_launches": K,
-        "e2e": e2e, "cpu_baseline": cpu, "breakdown": breakdown,
+        "config": config_block(wl0, world),
+        "roofline": head["roofline"], "clocks": head["clocks"], "gpu_launches": head["K"],
+        "e2e": head.get("e2e"), "cpu_baseline": head.get("cpu_baseline"),
+        "breakdown": head.get("breakdown"), "per_config": per_config,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -438,14 +598,19 @@ def run_ours(args):
     return 0
 
 
-def measure_e2e(cp, wl, o_h, m_h, s_h, sets, stream, dev, K, Wm, barrier, world, dist, tdt):
+def measure_e2e(cp, wl, inp, stream, dev, K, Wm, barrier, world):
     """Same metric, end to end through the public API with host buffers: every
     step copies its inputs from pinned host memory to the device, runs the
     fused call, and copies its outputs back to pinned host memory. Consecutive
     steps are pipelined on two streams over two device buffer sets, so step
     i+1's upload overlaps step i's download on the full-duplex host link."""
     import torch
-    nb = min(2, len(sets))
+    sets = list(inp.sets)
+    if len(sets) < 2:
+        # a second device buffer set, so that step i+1's upload overlaps step i
+        sets.append(tuple(torch.empty_like(t) for t in sets[0]))
+    o_h, m_h, s_h = inp.o_h, inp.m_h, inp.s_h
+    nb = 2
     up = torch.cuda.Stream(dev)              # host -> device
     work = torch.cuda.Stream(dev)            # kernel, then device -> host
     ho = [torch.empty(sets[0][3].shape, dtype=torch.int16, pin_memory=True) for _ in range(nb)]
@@ -498,29 +663,86 @@ def measure_e2e(cp, wl, o_h, m_h, s_h, sets, stream, dev, K, Wm, barrier, world,
                                  "pipelined on two streams; bound by the host link"}
 
 
-def _time(fn, stream, reps=20):
-    """Median device time of one call: back-to-back calls, each bracketed by
-    events on the launching stream, one synchronisation at the end."""
+# --------------------------------------------------------------------------------------------
+# the Before/After comparison of the DCP pull request, with its paired protocol
+
+def paired_ab(base, cand, stream, warmup=10, blocks=8, samples=5, null_blocks=4):
+    """Paired, interleaved A/B of two callables in a fixed order.
+
+    The protocol of the DCP pull request ("Performance evidence"): warm-up
+    iterations of both arms; `blocks` paired blocks, each timing `samples`
+    event-bracketed calls of the baseline and then `samples` of the candidate;
+    baseline-only null-control blocks (baseline against itself, same shape)
+    before and after; no samples added afterwards. A block's effect is the
+    relative improvement of the candidate's median over the baseline's. The
+    noise floor is the median absolute effect of the null-control blocks. The
+    rule fixed before measuring: positive if at least 75 % of the paired blocks
+    favour the candidate and the median paired improvement exceeds
+    max(1 %, 2 x noise floor); a regression under the mirror-image rule;
+    otherwise neutral."""
     import torch
-    for i in range(3):
-        fn(i)
+
+    def timed(fn, k):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(samples)]
+        hold_device(stream, 2.0)
+        for i in range(samples):
+            ev[i][0].record(stream)
+            fn(k * samples + i)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ev]
+
+    def block(a_fn, b_fn, k):
+        ta = statistics.median(timed(a_fn, k))
+        tb = statistics.median(timed(b_fn, k))
+        return ta, tb, (ta - tb) / ta
+
+    for i in range(warmup):
+        base(i)
+        cand(i)
     torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(reps)]
-    for i in range(reps):
-        ev[i][0].record(stream)
-        fn(i)
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    return statistics.median(a.elapsed_time(b) for a, b in ev)
+    pre = [block(base, base, k) for k in range(null_blocks)]
+    main = [block(base, cand, k) for k in range(blocks)]
+    post = [block(base, base, k) for k in range(null_blocks)]
+    rec = {"baseline_median_us": round(1e3 * statistics.median(a for a, _, _ in main), 3),
+           "candidate_median_us": round(1e3 * statistics.median(b for _, b, _ in main), 3)}
+    rec.update(ab_decision([e for _, _, e in main], [e for _, _, e in pre + post]))
+    rec["protocol"] = ("%d warm-ups; %d paired blocks x %d samples per arm, baseline first; "
+                       "%d + %d baseline-only null-control blocks before and after"
+                       % (warmup, blocks, samples, null_blocks, null_blocks))
+    return rec
 
 
-def measure_breakdown(cp, wl, sets, stream, dev, peak, tdt):
+def ab_decision(effects, null_effects):
+    """The decision rule of the paired A/B. `effects` are the paired blocks'
+    relative improvements of the candidate (positive: candidate faster),
+    `null_effects` those of the baseline-only null-control blocks."""
+    blocks = len(effects)
+    noise = statistics.median(abs(e) for e in null_effects)
+    effect = statistics.median(effects)
+    favour = sum(1 for e in effects if e > 0)
+    thresh = max(0.01, 2 * noise)
+    if favour >= 0.75 * blocks and effect > thresh:
+        verdict = "positive"
+    elif blocks - favour >= 0.75 * blocks and -effect > thresh:
+        verdict = "regression"
+    else:
+        verdict = "neutral"
+    return {"paired_median_effect": round(effect, 5),
+            "blocks_favouring_candidate": "%d/%d" % (favour, blocks),
+            "noise_floor": round(noise, 5), "threshold": round(thresh, 5), "verdict": verdict}
+
+
+def measure_breakdown(cp, wl, sets, stream, dev, peak):
     """Per-kernel times of the unfused path (and the Ulysses transforms on the
-    Ulysses workload), each against its own algorithmic bytes. Inputs rotate
-    over the device sets as in the timed region."""
+    Ulysses workload), each against its own algorithmic bytes, with the
+    Before/After A/B of the pack. Inputs rotate over the device sets as in the
+    timed region. Each figure is the median (p10, p90 beside it) of 20
+    separately event-bracketed launches."""
     import torch
     W, T, H, D, Hc = wl.W, wl.T, wl.H, wl.D, wl.Hc
+    tdt = sets[0][0].dtype
     n = len(sets)
     # two packet buffers alternate (L2 rotation) unless one alone exceeds L2 many times
     nb = 2 if W * T * H * D * 2 < 2e9 else 1
@@ -529,14 +751,12 @@ def measure_breakdown(cp, wl, sets, stream, dev, peak, tdt):
     rv = [(torch.empty_like(pk[0][0]), torch.empty_like(pk[0][1])) for _ in range(nb)]
     res = {}
 
-    def rec(name, ms, nbytes):
-        gbs = nbytes / (ms * 1e-3) / 1e9
-        res[name] = {"us": round(ms * 1e3, 2), "bytes": nbytes, "GB/s": round(gbs, 1),
-                     "frac": round(gbs / peak, 4)}
+    def rec(name, fn, nbytes, reps=20):
+        res[name] = launch_stats(time_launches(fn, stream, reps), nbytes, peak)
 
-    rec("pack", _time(lambda i: cp.cp_pack_lse(*sets[i % n][:3], pkt_o=pk[i % nb][0],
-                                               pkt_lse=pk[i % nb][1], stream=stream), stream),
-        wl.pack_bytes())
+    def pack(i):
+        cp.cp_pack_lse(*sets[i % n][:3], pkt_o=pk[i % nb][0], pkt_lse=pk[i % nb][1], stream=stream)
+    rec("pack", pack, wl.pack_bytes())
     rows = W * T * H
     # the Before pipeline of the DCP pull request: materialize LSE, then pack from it
     lse_buf = torch.empty((W, T, H), dtype=torch.float32, device=dev)
@@ -546,30 +766,30 @@ def measure_breakdown(cp, wl, sets, stream, dev, peak, tdt):
         cp.cp_lse_materialize(mi, si, lse=lse_buf, stream=stream)
         cp.cp_pack_from_lse(oi, lse_buf, pkt_o=pk[i % nb][0], pkt_lse=pk[i % nb][1], stream=stream)
     legacy_bytes = rows * (8 + 4) + rows * (2 * D * 2 + 4 + 4)
-    rec("legacy_pack", _time(legacy, stream), legacy_bytes)
+    rec("legacy_pack", legacy, legacy_bytes)
     res["legacy_over_pack"] = round(res["legacy_pack"]["us"] / res["pack"]["us"], 3)
+    res["legacy_ab"] = paired_ab(legacy, pack, stream)
     del lse_buf
 
     def perm(i):
         cp.cp_a2a_local_permute(pk[i % nb][0], W, recv=rv[i % nb][0], stream=stream)
         cp.cp_a2a_local_permute(pk[i % nb][1], W, recv=rv[i % nb][1], stream=stream)
-    rec("permute", _time(perm, stream), 2 * rows * (D * 2 + 4))
+    rec("permute", perm, 2 * rows * (D * 2 + 4))
     outs = [(torch.empty((W, T, Hc, D), dtype=tdt, device=dev),
              torch.empty((W, T, Hc), dtype=torch.float32, device=dev)) for _ in range(nb)]
-    rec("combine", _time(lambda i: cp.cp_lse_combine(*rv[i % nb], out=outs[i % nb][0],
-                                                     out_lse=outs[i % nb][1], stream=stream),
-                         stream), wl.combine_bytes())
-    unfused_us = res["pack"]["us"] + res["permute"]["us"] + res["combine"]["us"]
-    res["unfused_total_us"] = round(unfused_us, 2)
+    rec("combine", lambda i: cp.cp_lse_combine(*rv[i % nb], out=outs[i % nb][0],
+                                               out_lse=outs[i % nb][1], stream=stream),
+        wl.combine_bytes())
+    res["unfused_total_us"] = round(res["pack"]["us"] + res["permute"]["us"] + res["combine"]["us"], 2)
     del pk, rv, outs
     if T % W == 0:
         # the fused exchange of token chunks (same bytes, output in source order)
         touts = [(torch.empty((W, T // W, H, D), dtype=tdt, device=dev),
                   torch.empty((W, T // W, H), dtype=torch.float32, device=dev)) for _ in range(nb)]
         rec("fused_token_chunks",
-            _time(lambda i: cp.cp_pack_permute_combine_fused(*sets[i % n][:3], out=touts[i % nb][0],
-                                                             out_lse=touts[i % nb][1], scatter_dim=0,
-                                                             stream=stream), stream),
+            lambda i: cp.cp_pack_permute_combine_fused(*sets[i % n][:3], out=touts[i % nb][0],
+                                                       out_lse=touts[i % nb][1], scatter_dim=0,
+                                                       stream=stream),
             wl.fused_bytes())
         del touts
     # context for the fused share at this size: a plain device-to-device copy
@@ -578,20 +798,22 @@ def measure_breakdown(cp, wl, sets, stream, dev, peak, tdt):
     half = wl.fused_bytes() // 32 * 16
     srcs = [s[0].reshape(-1).view(torch.uint8)[:half] for s in sets]
     dsts = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(nb)]
-    rec("copy_same_bytes", _time(lambda i: dsts[i % nb].copy_(srcs[i % n]), stream), 2 * half)
+    rec("copy_same_bytes", lambda i: dsts[i % nb].copy_(srcs[i % n]), 2 * half)
     del srcs, dsts
     if wl.name == "ulysses":
         S_l = T // W
         xs = [torch.empty((W, 3, S_l, H, D), dtype=tdt, device=dev).normal_() for _ in range(2)]
         ys = [torch.empty((W, 3, T, Hc, D), dtype=tdt, device=dev) for _ in range(2)]
-        nb = 2 * xs[0].numel() * 2
-        rec("ulysses_seq2head", _time(lambda i: cp.ulysses_seq2head(xs[i % 2], out=ys[i % 2],
-                                                                    stream=stream), stream), nb)
+        rec("ulysses_seq2head", lambda i: cp.ulysses_seq2head(xs[i % 2], out=ys[i % 2],
+                                                              stream=stream),
+            2 * xs[0].numel() * 2)
+        del xs, ys
         hs = [torch.empty((W, 1, T, Hc, D), dtype=tdt, device=dev).normal_() for _ in range(2)]
         gs = [torch.empty((W, 1, S_l, H, D), dtype=tdt, device=dev) for _ in range(2)]
-        nb = 2 * hs[0].numel() * 2
-        rec("ulysses_head2seq", _time(lambda i: cp.ulysses_head2seq(hs[i % 2], out=gs[i % 2],
-                                                                    stream=stream), stream), nb)
+        rec("ulysses_head2seq", lambda i: cp.ulysses_head2seq(hs[i % 2], out=gs[i % 2],
+                                                              stream=stream),
+            2 * hs[0].numel() * 2)
+        del hs, gs
     torch.cuda.synchronize()
     return res
 

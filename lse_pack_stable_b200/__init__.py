@@ -112,6 +112,40 @@ def _dense(t: torch.Tensor, name: str) -> None:
         raise ValueError("%s must be contiguous" % name)
 
 
+def _expect(t: torch.Tensor, name: str, shape, dtype, device: torch.device) -> None:
+    """The C layer derives every extent from the sizes it is given, so a tensor
+    of another shape, type or device would be read or written out of bounds:
+    refuse it here."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if t.dtype != dtype:
+        raise ValueError("%s has dtype %s, expected %s" % (name, t.dtype, dtype))
+    if t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+
+
+def _payload(t: torch.Tensor, name: str, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.dim() != ndim:
+        raise ValueError("%s must have %d dimensions, got shape %s" % (name, ndim, tuple(t.shape)))
+    _dtype(t)
+
+
+def _stats(o: torch.Tensor, smax: torch.Tensor, ssum: torch.Tensor) -> None:
+    W, T, H = o.shape[:3]
+    _expect(smax, "smax", (W, T, H), torch.float32, o.device)
+    _expect(ssum, "ssum", (W, T, H), torch.float32, o.device)
+
+
+def _split(n: int, W: int, what: str) -> int:
+    if W < 1 or n % W != 0:
+        raise ValueError("%s = %d is not a multiple of W = %d" % (what, n, W))
+    return n // W
+
+
 def abi_version() -> int:
     return _lib.cp_abi_version()
 
@@ -120,18 +154,27 @@ def last_error() -> str:
     return _lib.cp_last_error().decode()
 
 
+def _packet_shape(W: int, T: int, H: int, scatter_dim: int):
+    if scatter_dim == 1:
+        return (W, W, T, _split(H, W, "H"))
+    if scatter_dim == 0:
+        return (W, W, _split(T, W, "T"), H)
+    raise ValueError("scatter_dim must be 0 (tokens) or 1 (heads), got %r" % (scatter_dim,))
+
+
 def cp_pack_lse(o: torch.Tensor, smax: torch.Tensor, ssum: torch.Tensor, scatter_dim: int = 1,
                 pkt_o: Optional[torch.Tensor] = None, pkt_lse: Optional[torch.Tensor] = None,
                 stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    _payload(o, "o", 4)
     W, T, H, D = o.shape
-    if scatter_dim == 1:
-        shape = (W, W, T, H // W)
-    else:
-        shape = (W, W, T // W, H)
+    _stats(o, smax, ssum)
+    shape = _packet_shape(W, T, H, scatter_dim)
     if pkt_o is None:
         pkt_o = torch.empty(shape + (D,), dtype=o.dtype, device=o.device)
     if pkt_lse is None:
         pkt_lse = torch.empty(shape, dtype=torch.float32, device=o.device)
+    _expect(pkt_o, "pkt_o", shape + (D,), o.dtype, o.device)
+    _expect(pkt_lse, "pkt_lse", shape, torch.float32, o.device)
     _dense(pkt_o, "pkt_o")
     _dense(pkt_lse, "pkt_lse")
     _check(_lib.cp_pack_lse(_ptr(o), _strides3(o), _ptr(smax), _strides3(smax), _ptr(ssum),
@@ -143,9 +186,14 @@ def cp_pack_lse(o: torch.Tensor, smax: torch.Tensor, ssum: torch.Tensor, scatter
 def cp_lse_materialize(smax: torch.Tensor, ssum: torch.Tensor, lse: Optional[torch.Tensor] = None,
                        stream=None) -> torch.Tensor:
     """Legacy first step: LSE [W, T, H] float32 from softmax max/sum."""
+    if not isinstance(smax, torch.Tensor) or smax.dim() != 3:
+        raise ValueError("smax must be a [W, T, H] tensor")
     W, T, H = smax.shape
+    _expect(smax, "smax", (W, T, H), torch.float32, smax.device)
+    _expect(ssum, "ssum", (W, T, H), torch.float32, smax.device)
     if lse is None:
         lse = torch.empty((W, T, H), dtype=torch.float32, device=smax.device)
+    _expect(lse, "lse", (W, T, H), torch.float32, smax.device)
     _dense(lse, "lse")
     _check(_lib.cp_lse_materialize(_ptr(smax), _strides3(smax), _ptr(ssum), _strides3(ssum), W, T,
                                    H, _ptr(lse), _stream(stream)))
@@ -156,12 +204,16 @@ def cp_pack_from_lse(o: torch.Tensor, lse: torch.Tensor, scatter_dim: int = 1,
                      pkt_o: Optional[torch.Tensor] = None, pkt_lse: Optional[torch.Tensor] = None,
                      stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Legacy pack: the packet of cp_pack_lse, its LSE region copied from `lse`."""
+    _payload(o, "o", 4)
     W, T, H, D = o.shape
-    shape = (W, W, T, H // W) if scatter_dim == 1 else (W, W, T // W, H)
+    _expect(lse, "lse", (W, T, H), torch.float32, o.device)
+    shape = _packet_shape(W, T, H, scatter_dim)
     if pkt_o is None:
         pkt_o = torch.empty(shape + (D,), dtype=o.dtype, device=o.device)
     if pkt_lse is None:
         pkt_lse = torch.empty(shape, dtype=torch.float32, device=o.device)
+    _expect(pkt_o, "pkt_o", shape + (D,), o.dtype, o.device)
+    _expect(pkt_lse, "pkt_lse", shape, torch.float32, o.device)
     _dense(pkt_o, "pkt_o")
     _dense(pkt_lse, "pkt_lse")
     _check(_lib.cp_pack_from_lse(_ptr(o), _strides3(o), _ptr(lse), _strides3(lse), W, T, H, D,
@@ -178,6 +230,9 @@ def cp_a2a_local_permute(send: torch.Tensor, W: int, recv: Optional[torch.Tensor
     _dense(send, "send")
     _dense(recv, "recv")
     nbytes = send.numel() * send.element_size()
+    if recv.numel() * recv.element_size() != nbytes or recv.device != send.device:
+        raise ValueError("recv must have the bytes (%d) and device (%s) of send"
+                         % (nbytes, send.device))
     if nbytes % (W * W) != 0:
         raise ValueError("send bytes (%d) are not W*W equal blocks" % nbytes)
     _check(_lib.cp_a2a_local_permute(_ptr(send), _ptr(recv), W, nbytes // (W * W),
@@ -189,11 +244,17 @@ def cp_lse_combine(recv_o: torch.Tensor, recv_lse: torch.Tensor,
                    out: Optional[torch.Tensor] = None, out_lse: Optional[torch.Tensor] = None,
                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """recv_o [W, W, T, Hc, D], recv_lse [W, W, T, Hc] -> out [W, T, Hc, D], out_lse [W, T, Hc]."""
+    _payload(recv_o, "recv_o", 5)
     W, W2, T, Hc, D = recv_o.shape
+    if W2 != W:
+        raise ValueError("recv_o must be [W, W, T, Hc, D], got %s" % (tuple(recv_o.shape),))
+    _expect(recv_lse, "recv_lse", (W, W, T, Hc), torch.float32, recv_o.device)
     if out is None:
         out = torch.empty((W, T, Hc, D), dtype=recv_o.dtype, device=recv_o.device)
     if out_lse is None:
         out_lse = torch.empty((W, T, Hc), dtype=torch.float32, device=recv_o.device)
+    _expect(out, "out", (W, T, Hc, D), recv_o.dtype, recv_o.device)
+    _expect(out_lse, "out_lse", (W, T, Hc), torch.float32, recv_o.device)
     for t, n in ((recv_o, "recv_o"), (recv_lse, "recv_lse"), (out, "out"), (out_lse, "out_lse")):
         _dense(t, n)
     _check(_lib.cp_lse_combine(_ptr(recv_o), _ptr(recv_lse), W, T, Hc, D, _dtype(recv_o),
@@ -207,12 +268,16 @@ def cp_pack_permute_combine_fused(o: torch.Tensor, smax: torch.Tensor, ssum: tor
                                   stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Head chunks (scatter_dim=1): out [W, T, H/W, D], out_lse [W, T, H/W].
     Token chunks (scatter_dim=0): out [W, T/W, H, D], out_lse [W, T/W, H]."""
+    _payload(o, "o", 4)
     W, T, H, D = o.shape
-    shape = (W, T, H // W) if scatter_dim == 1 else (W, T // W, H)
+    _stats(o, smax, ssum)
+    shape = _packet_shape(W, T, H, scatter_dim)[1:]
     if out is None:
         out = torch.empty(shape + (D,), dtype=o.dtype, device=o.device)
     if out_lse is None:
         out_lse = torch.empty(shape, dtype=torch.float32, device=o.device)
+    _expect(out, "out", shape + (D,), o.dtype, o.device)
+    _expect(out_lse, "out_lse", shape, torch.float32, o.device)
     _dense(out, "out")
     _dense(out_lse, "out_lse")
     _check(_lib.cp_pack_permute_combine_fused(_ptr(o), _strides3(o), _ptr(smax), _strides3(smax),
@@ -225,9 +290,13 @@ def cp_pack_permute_combine_fused(o: torch.Tensor, smax: torch.Tensor, ssum: tor
 def ulysses_seq2head(x: torch.Tensor, out: Optional[torch.Tensor] = None,
                      stream=None) -> torch.Tensor:
     """x [W, B, S/W, H, D] (contiguous) -> [W, B, S, H/W, D]."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 5:
+        raise ValueError("x must be a [W, B, S/W, H, D] tensor")
     W, B, S_l, H, D = x.shape
+    shape = (W, B, S_l * W, _split(H, W, "H"), D)
     if out is None:
-        out = torch.empty((W, B, S_l * W, H // W, D), dtype=x.dtype, device=x.device)
+        out = torch.empty(shape, dtype=x.dtype, device=x.device)
+    _expect(out, "out", shape, x.dtype, x.device)
     _dense(x, "x")
     _dense(out, "out")
     _check(_lib.ulysses_seq2head(_ptr(x), _ptr(out), W, B, S_l, H, D, x.element_size(),
@@ -238,9 +307,13 @@ def ulysses_seq2head(x: torch.Tensor, out: Optional[torch.Tensor] = None,
 def ulysses_head2seq(x: torch.Tensor, out: Optional[torch.Tensor] = None,
                      stream=None) -> torch.Tensor:
     """x [W, B, S, Hc, D] (contiguous) -> [W, B, S/W, Hc*W, D]."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 5:
+        raise ValueError("x must be a [W, B, S, H/W, D] tensor")
     W, B, S, Hc, D = x.shape
+    shape = (W, B, _split(S, W, "S"), Hc * W, D)
     if out is None:
-        out = torch.empty((W, B, S // W, Hc * W, D), dtype=x.dtype, device=x.device)
+        out = torch.empty(shape, dtype=x.dtype, device=x.device)
+    _expect(out, "out", shape, x.dtype, x.device)
     _dense(x, "x")
     _dense(out, "out")
     _check(_lib.ulysses_head2seq(_ptr(x), _ptr(out), W, B, S // W, Hc * W, D, x.element_size(),

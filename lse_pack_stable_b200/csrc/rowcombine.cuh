@@ -41,41 +41,10 @@ namespace cplse {
 constexpr int kCombineThreads = CPLSE_COMBINE_THREADS;
 // 16-byte loads each lane keeps in flight in phase B (sets U below)
 constexpr int kLoadsInFlight = CPLSE_LOADS_IN_FLIGHT;
-#ifndef CPLSE_PREFETCH
-#define CPLSE_PREFETCH 0
-#endif
 constexpr unsigned kFull = 0xffffffffu;
 constexpr uint32_t kNegZero2 = 0x80008000u;   // two -0.0 payload elements
 
 enum { kModeFused = 0, kModeCombine = 1 };
-
-// Ask the L2 to fetch `bytes` (multiple of 16, 16-byte aligned) starting at p.
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-// L2 prefetch of chunk c's payload rows, one lane per rank: the rank-r rows of
-// a chunk are contiguous when the rows are dense (row stride D). Combine mode
-// stops at the end of the (dst, src) block the chunk starts in.
-template <int MODE>
-__device__ __forceinline__ void prefetch_chunk(const CombineArgs& a, int64_t c, int lane)
-{
-    if (!a.dense_rows || lane >= a.W) return;
-    const int64_t q0 = c * 32;
-    if (q0 >= a.rows) return;
-    int64_t q1 = q0 + 32 < a.rows ? q0 + 32 : a.rows;
-    int64_t base;
-    if (MODE == kModeFused) {
-        base = q0 * a.D + lane * a.rank_stride;
-    } else {
-        const int64_t j = q0 / a.N, n0 = q0 - j * a.N;
-        const int64_t n1 = n0 + (q1 - q0) < a.N ? n0 + (q1 - q0) : a.N;
-        q1 = q0 + (n1 - n0);
-        base = (j * a.W * a.N + n0) * a.D + lane * a.rank_stride;
-    }
-    prefetch_l2(a.src + base, (uint32_t)((q1 - q0) * a.D * 2));
-}
 
 // Phase A for one row: addresses and the W LSE values (-inf beyond W or q).
 template <int MODE, int WMAX>
@@ -146,13 +115,14 @@ rowcombine_kernel(const CombineArgs a)
     const int V = a.D >> 3;
     const int64_t rank_stride = a.rank_stride;
 
-#if CPLSE_PREFETCH
-    if (warp < nchunks) prefetch_chunk<MODE>(a, warp, lane);
-#endif
+    // Programmatic dependent launch, as in the shared-memory-staged kernel: the
+    // next kernel in the stream may be scheduled now, and this one reads
+    // nothing until the previous kernel has completed and its writes are
+    // visible.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
     for (int64_t c = warp; c < nchunks; c += nwarps) {
-#if CPLSE_PREFETCH >= 2
-        if (c + nwarps < nchunks) prefetch_chunk<MODE>(a, c + nwarps, lane);
-#endif
         // ---------------- phase A: lane owns row c*32 + lane
         const int64_t q = c * 32 + lane;
         const bool qv = q < a.rows;
@@ -262,6 +232,29 @@ rowcombine_kernel(const CombineArgs a)
     }
 }
 
+// Launch with programmatic stream serialization: back-to-back launches overlap
+// the next grid's scheduling with this one's drain. Every merge kernel opens
+// with griddepcontrol.wait, so none reads memory before the previous kernel in
+// the stream has completed.
+template <typename K>
+cudaError_t launch_pdl(K kern, unsigned blocks, int threads, int smem, cudaStream_t s,
+                       const CombineArgs& a)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 // Lanes per row and vectors per lane for a head dim of D elements (D % 8 == 0).
 struct RowShape {
     int G, VPL;
@@ -295,8 +288,7 @@ cudaError_t launch_rowcombine_inst(const CombineArgs& a, cudaStream_t s)
     const int64_t cap = (int64_t)per_sm * sm_count();
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    kern<<<(unsigned)blocks, kCombineThreads, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(kern, (unsigned)blocks, kCombineThreads, 0, s, a);
 }
 
 }  // namespace cplse

@@ -36,21 +36,7 @@ cudaError_t launch_async_inst(const CombineArgs& a, cudaStream_t s)
     const int64_t cap = (int64_t)per_sm * sm_count();
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    // programmatic stream serialization: back-to-back launches overlap the next
-    // grid's scheduling with this one's drain (the kernel waits on griddepcontrol)
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)blocks);
-    cfg.blockDim = dim3(kAsyncThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    return launch_pdl(kern, (unsigned)blocks, kAsyncThreads, smem, s, a);
 }
 
 // Shared-memory staging for up to 8 ranks; register staging from 16 ranks on,

@@ -59,12 +59,19 @@ TID_LSE = 0xC000        # direct LSE inputs for the combine-only cases
 
 
 def fill(seed: int, tid: int, dist: int, p0: float, p1: float, n: int = 0, start: int = 0,
-         idx: Optional[np.ndarray] = None, fmt: int = F32) -> np.ndarray:
-    """Draw n values (or one per entry of ``idx``) from stream (seed, tid)."""
+         idx: Optional[np.ndarray] = None, fmt: int = F32,
+         out: Optional[np.ndarray] = None) -> np.ndarray:
+    """Draw n values (or one per entry of ``idx``) from stream (seed, tid), into
+    ``out`` (a C-contiguous array of n elements of the format's type) if given."""
     if idx is not None:
         idx = np.ascontiguousarray(idx, dtype=np.uint64)
         n = idx.size
-    out = np.empty(n, dtype=_NP[fmt])
+    if out is None:
+        out = np.empty(n, dtype=_NP[fmt])
+    else:
+        if out.dtype != _NP[fmt] or out.size != n or not out.flags.c_contiguous:
+            raise ValueError("out must be C-contiguous %s with %d elements" % (_NP[fmt], n))
+        out = out.reshape(-1)
     if n:
         _lib.synth_fill(seed, tid, dist, p0, p1, start,
                         idx.ctypes.data if idx is not None else None, n, fmt, out.ctypes.data)
@@ -148,11 +155,14 @@ CONFIGS = {
 # ----------------------------------------------------------------------------------------------
 # partial outputs O_r[t][h][:]
 
-def o_block(wl: Workload, r: int, t0: int = 0, t1: Optional[int] = None) -> np.ndarray:
-    """O_r[t0:t1] as raw 16-bit payload, shape [t1-t0, H, D]."""
+def o_block(wl: Workload, r: int, t0: int = 0, t1: Optional[int] = None,
+            out: Optional[np.ndarray] = None) -> np.ndarray:
+    """O_r[t0:t1] as raw 16-bit payload, shape [t1-t0, H, D] (written into
+    ``out``, a C-contiguous uint16 array of that size, if given)."""
     t1 = wl.T if t1 is None else t1
     n = (t1 - t0) * wl.H * wl.D
-    v = fill(wl.seed, TID_O + r, NORMAL, 0.0, wl.o_sigma, n=n, start=t0 * wl.H * wl.D, fmt=wl.fmt)
+    v = fill(wl.seed, TID_O + r, NORMAL, 0.0, wl.o_sigma, n=n, start=t0 * wl.H * wl.D, fmt=wl.fmt,
+             out=out)
     return v.reshape(t1 - t0, wl.H, wl.D)
 
 

@@ -70,3 +70,36 @@ def test_reference_arm_under_torchrun_prints_one_line():
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["unit"] == "GB/s"
     assert rec["cpu_baseline"]["kind"] == "oracle" and rec["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_ab_decision_rule():
+    """The paired A/B's rule: positive needs >= 75 % of blocks for the
+    candidate AND a median improvement above max(1 %, 2 x noise floor)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    null = [0.004, -0.003, 0.002, -0.006]            # noise floor = median |e| = 0.0035
+    pos = bench.ab_decision([0.2, 0.21, 0.19, 0.2, 0.22, 0.18, 0.2, 0.2], null)
+    assert pos["verdict"] == "positive" and pos["blocks_favouring_candidate"] == "8/8"
+    assert pos["noise_floor"] == pytest.approx(0.0035) and pos["threshold"] == pytest.approx(0.01)
+    # 6/8 blocks (75 %) favour the candidate, median effect 1.5 % > 1 %: positive
+    assert bench.ab_decision([0.02, 0.02, 0.015, 0.015, 0.02, 0.015, -0.01, -0.01],
+                             null)["verdict"] == "positive"
+    # 5/8 favour the candidate: neutral however large the effect
+    assert bench.ab_decision([0.3, 0.3, 0.3, 0.3, 0.3, -0.1, -0.1, -0.1], null)["verdict"] == "neutral"
+    # a noisy floor raises the threshold: 3 % improvement against a 2 % floor (4 % bar)
+    assert bench.ab_decision([0.03] * 8, [0.02, -0.02, 0.02, -0.02])["verdict"] == "neutral"
+    # the mirror image is a regression
+    assert bench.ab_decision([-0.05] * 8, null)["verdict"] == "regression"
+
+
+def test_rotation_policy_is_a_function_of_the_workload():
+    """Both arms print the same config, so the L2 note cannot depend on the device."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    assert bench.rotation_sets(synth.CONFIGS["stress"]) == 1
+    assert bench.rotation_sets(synth.CONFIGS["mla"]) == 1
+    n = bench.rotation_sets(synth.CONFIGS["decode"])
+    assert n >= 2 and n * synth.CONFIGS["decode"].fused_bytes() >= 3 * bench.L2_BYTES
+    a = bench.config_block(synth.CONFIGS["decode"], 1)
+    assert a == bench.config_block(synth.CONFIGS["decode"], 1) and "l2" in a
