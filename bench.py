@@ -99,13 +99,34 @@ def l2_note(wl: synth.Workload) -> str:
             % (n, b / 1e6, n * b / 1e6))
 
 
+def workload_for(name: str, world: int) -> synth.Workload:
+    """The workload a run on `world` GPUs measures: on one GPU the configured
+    one, W ranks emulated; on N > 1 GPUs the same T, H, D and distributions
+    with W = N real ranks, rank r holding plane r (one per GPU)."""
+    wl = synth.CONFIGS[name]
+    if world == 1:
+        return wl
+    if wl.H % world:
+        raise SystemExit("%s: H = %d is not a multiple of %d GPUs" % (name, wl.H, world))
+    return synth.Workload(**{**wl.__dict__, "W": world})
+
+
 def config_block(wl: synth.Workload, world: int):
     """The workload's description; identical in both arms of the benchmark."""
-    return {"workload": "%s: W=%d simulated ranks, T=%d, H=%d, D=%d, %s payload, fp32 max/sum"
-                        % (wl.name, wl.W, wl.T, wl.H, wl.D, wl.dtype),
+    if world == 1:
+        return {"workload": "%s: W=%d simulated ranks, T=%d, H=%d, D=%d, %s payload, fp32 max/sum"
+                            % (wl.name, wl.W, wl.T, wl.H, wl.D, wl.dtype),
+                "W": wl.W, "T": wl.T, "H": wl.H, "D": wl.D, "payload_dtype": wl.dtype,
+                "global_batch": 1, "parallelism": "replicas1",
+                "bytes_per_call": wl.fused_bytes(), "l2": l2_note(wl)}
+    return {"workload": "%s shape across %d GPUs: W=%d real ranks (KV shard r on GPU r), T=%d, "
+                        "H=%d, D=%d, %s payload, fp32 max/sum; destination j combines head chunk j"
+                        % (wl.name, world, wl.W, wl.T, wl.H, wl.D, wl.dtype),
             "W": wl.W, "T": wl.T, "H": wl.H, "D": wl.D, "payload_dtype": wl.dtype,
-            "global_batch": world, "parallelism": "replicas%d" % world,
-            "bytes_per_call": wl.fused_bytes(), "l2": l2_note(wl)}
+            "global_batch": 1, "parallelism": "dcp%d" % world,
+            "bytes_per_call": wl.fused_bytes(),
+            "l2": "one set per rank, %.2f GB of planes per GPU (> 3x the L2)"
+                  % (wl.T * wl.H * (2 * wl.D + 8) / 1e9)}
 
 
 def reduce_max(values, world, device):
@@ -328,7 +349,7 @@ def run_reference(args):
     rank, _, world = env_rank()
     if rank != 0:
         return 0
-    wl = synth.CONFIGS[args.config]
+    wl = workload_for(args.config, world)
     steps, warm = max(1, args.steps), max(0, args.warmup)
     orc, fmt = _oracle_fmt(wl)
     o, m, s = sample_inputs(wl, min(wl.T, 16))
@@ -547,24 +568,29 @@ def run_ours(args):
     rank, local_rank, world = env_rank()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    peak, peak_kind = measured_peak()
     if world > 1:
+        # the communicator's own log stays on; no NVLink multicast (NVLS) objects
+        os.environ.setdefault("NCCL_DEBUG", "INFO")
+        os.environ.setdefault("NCCL_NVLS_ENABLE", "0")
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
+        try:
+            return run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind)
+        finally:
+            dist.destroy_process_group()
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        pass
 
-    wl0 = synth.CONFIGS[args.config]
-    wl = synth.Workload(**{**wl0.__dict__, "seed": wl0.seed + 1000 * rank})
+    wl = synth.CONFIGS[args.config]
     stream = torch.cuda.current_stream(dev)
-    peak, peak_kind = measured_peak()
 
-    head = measure_workload(cp, wl, dev, stream, args, world, barrier, peak, peak_kind, True)
+    head = measure_workload(cp, wl, dev, stream, args, 1, barrier, peak, peak_kind, True)
 
     per_config = None
     names = [] if args.per_config in ("", "none") else args.per_config.split(",")
-    if world == 1 and names:
+    if names:
         per_config = {}
         for name in names:
             if name == args.config:
@@ -585,16 +611,128 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "payload_dtype": wl.dtype,
         "data": "synthetic (seeded counter-based generator, the workload's shapes and distributions)",
-        "config": config_block(wl0, world),
+        "config": config_block(wl, 1),
         "roofline": head["roofline"], "clocks": head["clocks"], "gpu_launches": head["K"],
         "e2e": head.get("e2e"), "cpu_baseline": head.get("cpu_baseline"),
         "breakdown": head.get("breakdown"), "per_config": per_config,
     }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------------------------
+# N > 1 GPUs: the exchange across real ranks
+
+NVLINK_PEER_GBS = 770.0        # measured peer copy per direction on this machine's B200s
+
+
+def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
+    """One rank per GPU, W = N. Each step is the whole exchange for every
+    destination at once: rank j pulls head chunk j of every rank's planes
+    (PullExchange: barrier, cp_pull_combine, barrier). The NCCL path (pack,
+    two all-to-alls, combine) is timed the same way as the baseline, and the
+    two must agree bit for bit on every rank."""
+    import torch
+    import torch.distributed as dist
+    from lse_pack_stable_b200.exchange import A2aExchange, PullExchange
+
+    wl = workload_for(args.config, world)
+    T, H, D, Hc = wl.T, wl.H, wl.D, wl.H // world
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float16
+    stream = torch.cuda.current_stream(dev)
+
+    # this rank's plane of the N-rank workload, generated on the host (pinned:
+    # the end-to-end leg uploads from there)
+    o_h = torch.empty((T, H, D), dtype=torch.int16, pin_memory=True)
+    on = o_h.numpy().view(np.uint16)
+    tb = max(1, (256 << 20) // (H * D * 2))
+    for t0 in range(0, T, tb):
+        synth.o_block(wl, rank, t0, min(T, t0 + tb), out=on[t0:min(T, t0 + tb)])
+    mr, sr = synth.stats_block(wl, rank)
+    m_h = torch.from_numpy(mr).pin_memory()
+    s_h = torch.from_numpy(sr).pin_memory()
+
+    pull = PullExchange(T, H, D, tdt, dev)
+    pull.o.view(torch.int16).copy_(o_h)
+    pull.smax.copy_(m_h)
+    pull.ssum.copy_(s_h)
+    a2a = A2aExchange(T, H, D, tdt, dev)
+    out_p = torch.empty((T, Hc, D), dtype=tdt, device=dev)
+    lse_p = torch.empty((T, Hc), dtype=torch.float32, device=dev)
+    out_a = torch.empty_like(out_p)
+    lse_a = torch.empty_like(lse_p)
+
+    def barrier():
+        dist.barrier()
+
+    K, Wm = max(1, args.steps), max(3, args.warmup)
+    # the two paths agree bit for bit (checked on every rank, then reduced)
+    pull(out_p, lse_p)
+    a2a(pull.o, pull.smax, pull.ssum, out_a, lse_a)
+    torch.cuda.synchronize()
+    same = torch.tensor([float(torch.equal(out_p.view(torch.int16), out_a.view(torch.int16))
+                               and torch.equal(lse_p.view(torch.int32), lse_a.view(torch.int32)))],
+                        device=dev)
+    dist.all_reduce(same, op=dist.ReduceOp.MIN)
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    pull_ms = time_back_to_back(lambda i: pull(out_p, lse_p), stream, K, Wm, barrier)
+    a2a_ms = time_back_to_back(lambda i: a2a(pull.o, pull.smax, pull.ssum, out_a, lse_a), stream,
+                               K, Wm, barrier)
+    clocks.stop()
+    pull_ms, a2a_ms = reduce_max([pull_ms, a2a_ms], world, dev)
+    bytes_per_call = wl.fused_bytes()                 # every rank's reads and writes together
+    value = bytes_per_call * K / (pull_ms * 1e-3) / 1e9
+    # NVLink roofline: each destination reads (W-1) of its W contributions from peers
+    remote = (world - 1) * T * Hc * (2 * D + 8)
+    achieved = remote / (pull_ms / K * 1e-3) / 1e9
+
+    # end to end through the public API: upload this rank's plane into its
+    # shared buffers, exchange, download this destination's rows
+    ho = torch.empty((T, Hc, D), dtype=torch.int16, pin_memory=True)
+    hl = torch.empty((T, Hc), dtype=torch.float32, pin_memory=True)
+
+    def e2e_step(i):
+        pull.o.view(torch.int16).copy_(o_h, non_blocking=True)
+        pull.smax.copy_(m_h, non_blocking=True)
+        pull.ssum.copy_(s_h, non_blocking=True)
+        pull(out_p, lse_p)
+        ho.copy_(out_p.view(torch.int16), non_blocking=True)
+        hl.copy_(lse_p, non_blocking=True)
+    ke = max(3, min(K, 20))
+    e2e_ms = reduce_max([time_back_to_back(e2e_step, stream, ke, 3, barrier)], world, dev)[0]
+    h2d = o_h.numel() * 2 + m_h.numel() * 4 + s_h.numel() * 4
+    d2h = ho.numel() * 2 + hl.numel() * 4
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": Wm, "ms_per_step": round(pull_ms / K, 5),
+        "us_per_call": round(pull_ms / K * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "payload_dtype": wl.dtype,
+        "data": "synthetic (seeded counter-based generator, the workload's shapes and distributions)",
+        "config": config_block(wl, world),
+        "roofline": {"bound": "nvlink", "achieved": round(achieved, 2), "peak": NVLINK_PEER_GBS,
+                     "unit": "GB/s", "frac": round(achieved / NVLINK_PEER_GBS, 4),
+                     "traffic": None, "kernel": "pull_combine_kernel (plain loads over NVLink)",
+                     "peak_source": "measured peer copy per direction on this pool (770 GB/s)",
+                     "nvlink_bytes_per_rank_per_call": remote},
+        "clocks": clocks.summary(), "gpu_launches": K,
+        "e2e": {"value": round(bytes_per_call * ke / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world,
+                "ms_per_step": round(e2e_ms / ke, 4), "steps": ke},
+        "exchange": {"pull_equals_a2a": bool(same.item() == 1.0),
+                     "a2a_us_per_call": round(a2a_ms / K * 1e3, 3),
+                     "a2a_GB/s": round(bytes_per_call * K / (a2a_ms * 1e-3) / 1e9, 2),
+                     "a2a_path": "cp_pack_lse_rank -> NCCL all-to-all x2 -> cp_lse_combine_rank",
+                     "hbm_peak_GB/s": peak, "hbm_peak_source": peak_source(peak_kind)},
+        "cpu_baseline": None, "breakdown": None, "per_config": None,
+    }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    torch.cuda.synchronize()
+    pull.close()
     return 0
 
 

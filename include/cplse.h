@@ -55,7 +55,7 @@ extern "C" {
 #define CPLSE_API
 #endif
 
-#define CPLSE_ABI_VERSION 2
+#define CPLSE_ABI_VERSION 3
 #define CPLSE_MAX_W 32     /* simulated ranks per call */
 #define CPLSE_MAX_D 1024   /* head dim, elements */
 
@@ -174,6 +174,95 @@ CPLSE_API cp_status cp_pack_permute_combine_fused(const void* o, cp_strides3 so,
                                         cp_strides3 sm, const float* ssum, cp_strides3 ss, int W,
                                         int64_t T, int H, int D, cp_dtype dt, int scatter_dim,
                                         void* out, float* out_lse, void* stream);
+
+/*
+ * ---- One process per GPU: the exchange across W real ranks ----------------
+ *
+ * [DCP] The pipeline's all-to-all is a real collective when every rank is its
+ * own GPU: rank r holds the partial output of KV shard r (o [T][H][D] and its
+ * max/sum [T][H]); destination j receives head chunk j (or token chunk j) of
+ * every rank and combines it. Two ways to run it on B200:
+ *   a2a:  cp_pack_lse_rank -> an all-to-all of both packet regions (NCCL,
+ *         equal W-way splits) -> cp_lse_combine_rank;
+ *   pull: cp_pull_combine, one kernel per destination that loads the rows it
+ *         merges from every rank's o/max/sum where they live (peer memory
+ *         mapped into this process), so that no packet exists anywhere.
+ * All three give, on rank j, destination j's block of
+ * cp_pack_permute_combine_fused's output for the same W planes, bit for bit.
+ */
+
+/*
+ * Mapping another rank's buffers into this process for cp_pull_combine (CUDA
+ * IPC of plain device memory; no multicast, no fabric handles). The owner
+ * exports the address of a buffer it allocated with cudaMalloc (a caching
+ * allocator's block is fine: the handle names the whole allocation and the
+ * offset locates the buffer in it); the handle is plain bytes that the caller
+ * moves to the other processes of the same node. A reader imports it with its
+ * own device current: the owner's memory becomes addressable by the reader's
+ * kernels (peer access is enabled as needed). `base` is what cp_ipc_close
+ * takes once the reader is done; the owner must keep the buffer allocated
+ * until every reader has closed it. A handle cannot be imported by the
+ * process that exported it (CP_ERR_CUDA).
+ */
+typedef struct cp_ipc_handle {
+    unsigned char handle[64];   /* cudaIpcMemHandle_t of the allocation */
+    int64_t offset;             /* bytes from the allocation's start to the buffer */
+    int64_t alloc_bytes;        /* size of the allocation */
+    int32_t device;             /* the owner's device ordinal */
+    int32_t reserved;
+} cp_ipc_handle;
+
+CPLSE_API cp_status cp_ipc_export(const void* p, cp_ipc_handle* h);
+CPLSE_API cp_status cp_ipc_import(const cp_ipc_handle* h, void** base, void** p);
+CPLSE_API cp_status cp_ipc_close(void* base);
+
+/*
+ * [DCP] After pipeline, one real rank: the pack of cp_pack_lse for a single
+ * source plane. o [T][H][D] (strides so.t, so.h; so.r ignored), smax / ssum
+ * [T][H] fp32 (strides .t, .h; .r ignored). W is the number of destination
+ * ranks. Writes this rank's send packet, destination-major:
+ *   scatter_dim 1: pkt_o [W_dst][T][Hc][D], pkt_lse [W_dst][T][Hc]
+ *   scatter_dim 0: pkt_o [W_dst][T/W][H][D], pkt_lse [W_dst][T/W][H]
+ * equal to plane r of cp_pack_lse's packet for the same W planes. Each
+ * region splits into W equal contiguous blocks, one per destination, as an
+ * all-to-all with equal splits expects.
+ */
+CPLSE_API cp_status cp_pack_lse_rank(const void* o, cp_strides3 so, const float* smax,
+                                     cp_strides3 sm, const float* ssum, cp_strides3 ss, int W,
+                                     int64_t T, int H, int D, cp_dtype dt, int scatter_dim,
+                                     void* pkt_o, float* pkt_lse, void* stream);
+
+/*
+ * [DCP] The stable combine on one real destination rank, after the
+ * all-to-all: recv_o [W_src][N][D], recv_lse [W_src][N] (N = T*Hc rows; for
+ * token chunks pass T/W as T and H as Hc) -> out [N][D], out_lse [N]. Same
+ * rule and same bits as cp_lse_combine for one destination.
+ */
+CPLSE_API cp_status cp_lse_combine_rank(const void* recv_o, const float* recv_lse, int W,
+                                        int64_t T, int Hc, int D, cp_dtype dt, void* out,
+                                        float* out_lse, void* stream);
+
+/*
+ * [DCP] pack -> all-to-all -> combine for destination `dst` of W real ranks,
+ * in one kernel on dst's GPU, pulling each source row over NVLink.
+ *   o, smax, ssum  HOST arrays of W device addresses: rank r's o [T][H][D]
+ *                  and max/sum [T][H] planes. Each address must be usable by
+ *                  the current device: its own memory, or a peer's mapped into
+ *                  this process (CUDA IPC) with peer access between the two.
+ *                  Every plane has the layout given by so / sm / ss (.t, .h;
+ *                  .r ignored).
+ *   scatter_dim 1: out [T][Hc][D], out_lse [T][Hc]: heads dst*Hc .. of every token
+ *   scatter_dim 0: out [T/W][H][D], out_lse [T/W][H]: tokens dst*T/W .. with all heads
+ * The kernel reads the planes with ordinary 16-byte loads (no bulk or
+ * multicast copies) and waits for nothing: the caller orders it after every
+ * rank's writes to its planes and before any rank overwrites them again (a
+ * stream-ordered barrier such as a one-element all-reduce on both sides).
+ */
+CPLSE_API cp_status cp_pull_combine(const void* const* o, cp_strides3 so,
+                                    const float* const* smax, cp_strides3 sm,
+                                    const float* const* ssum, cp_strides3 ss, int W, int64_t T,
+                                    int H, int D, cp_dtype dt, int scatter_dim, int dst,
+                                    void* out, float* out_lse, void* stream);
 
 /*
  * [ULY] all_to_all_4D(x, scatter_dim=2, gather_dim=1), W ranks on one GPU:

@@ -19,7 +19,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from typing import Optional, Tuple
+from typing import Optional, Sequence, Tuple
 
 import torch
 
@@ -39,8 +39,9 @@ STATUS_NAMES = {0: "CP_OK", -1: "CP_ERR_ARG", -2: "CP_ERR_SHAPE", -3: "CP_ERR_AL
                 -4: "CP_ERR_ALIAS", -5: "CP_ERR_UNSUPPORTED", -6: "CP_ERR_CUDA"}
 EXPORTS = ("cp_abi_version", "cp_last_error", "cp_pack_lse", "cp_lse_materialize",
            "cp_pack_from_lse", "cp_a2a_local_permute",
-           "cp_lse_combine", "cp_pack_permute_combine_fused", "ulysses_seq2head",
-           "ulysses_head2seq")
+           "cp_lse_combine", "cp_pack_permute_combine_fused", "cp_pack_lse_rank",
+           "cp_lse_combine_rank", "cp_pull_combine", "cp_ipc_export", "cp_ipc_import",
+           "cp_ipc_close", "ulysses_seq2head", "ulysses_head2seq")
 
 
 class Strides3(ctypes.Structure):
@@ -50,7 +51,7 @@ class Strides3(ctypes.Structure):
 _p, _i, _i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
 _lib.cp_abi_version.argtypes = []
 _lib.cp_abi_version.restype = _i
-ABI_VERSION = 2           # include/cplse.h CPLSE_ABI_VERSION this binding marshals for
+ABI_VERSION = 3           # include/cplse.h CPLSE_ABI_VERSION this binding marshals for
 if _lib.cp_abi_version() != ABI_VERSION:
     raise ImportError("libcplse.so has ABI version %d, this binding needs %d: rebuild it with "
                       "`python lse_pack_stable_b200/build.py`" % (_lib.cp_abi_version(), ABI_VERSION))
@@ -64,11 +65,30 @@ _lib.cp_a2a_local_permute.argtypes = [_p, _p, _i, _i64, _p]
 _lib.cp_lse_combine.argtypes = [_p, _p, _i, _i64, _i, _i, _i, _p, _p, _p]
 _lib.cp_pack_permute_combine_fused.argtypes = [_p, Strides3, _p, Strides3, _p, Strides3, _i, _i64,
                                                _i, _i, _i, _i, _p, _p, _p]
+_lib.cp_pack_lse_rank.argtypes = [_p, Strides3, _p, Strides3, _p, Strides3, _i, _i64, _i, _i, _i,
+                                  _i, _p, _p, _p]
+_lib.cp_lse_combine_rank.argtypes = [_p, _p, _i, _i64, _i, _i, _i, _p, _p, _p]
+_lib.cp_pull_combine.argtypes = [_p, Strides3, _p, Strides3, _p, Strides3, _i, _i64, _i, _i, _i,
+                                 _i, _i, _p, _p, _p]
+
+
+class IpcHandle(ctypes.Structure):
+    """cp_ipc_handle of include/cplse.h."""
+    _fields_ = [("handle", ctypes.c_ubyte * 64), ("offset", ctypes.c_int64),
+                ("alloc_bytes", ctypes.c_int64), ("device", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+_lib.cp_ipc_export.argtypes = [_p, ctypes.POINTER(IpcHandle)]
+_lib.cp_ipc_import.argtypes = [ctypes.POINTER(IpcHandle), ctypes.POINTER(ctypes.c_void_p),
+                               ctypes.POINTER(ctypes.c_void_p)]
+_lib.cp_ipc_close.argtypes = [_p]
 _lib.ulysses_seq2head.argtypes = [_p, _p, _i, _i, _i64, _i, _i, _i, _p]
 _lib.ulysses_head2seq.argtypes = [_p, _p, _i, _i, _i64, _i, _i, _i, _p]
 for _f in ("cp_pack_lse", "cp_lse_materialize", "cp_pack_from_lse", "cp_a2a_local_permute",
-           "cp_lse_combine",
-           "cp_pack_permute_combine_fused", "ulysses_seq2head", "ulysses_head2seq"):
+           "cp_lse_combine", "cp_pack_permute_combine_fused", "cp_pack_lse_rank",
+           "cp_lse_combine_rank", "cp_pull_combine", "cp_ipc_export", "cp_ipc_import",
+           "cp_ipc_close", "ulysses_seq2head", "ulysses_head2seq"):
     getattr(_lib, _f).restype = _i
 
 
@@ -83,7 +103,7 @@ def _check(status: int) -> None:
         raise CplseError(status, _lib.cp_last_error().decode())
 
 
-def _dtype(t: torch.Tensor) -> int:
+def _dtype(t) -> int:
     if t.dtype == torch.bfloat16:
         return CP_BF16
     if t.dtype == torch.float16:
@@ -285,6 +305,121 @@ def cp_pack_permute_combine_fused(o: torch.Tensor, smax: torch.Tensor, ssum: tor
                                               scatter_dim, _ptr(out), _ptr(out_lse),
                                               _stream(stream)))
     return out, out_lse
+
+
+# ---- one process per GPU: the exchange across W real ranks ------------------------------------
+
+def _strides_plane(t) -> Strides3:
+    """Strides of one rank's [T, H] or [T, H, D] plane (the rank stride is unused)."""
+    st = t.stride()
+    if t.dim() == 3 and st[2] != 1:
+        raise ValueError("the head dim (last) of o must be contiguous")
+    return Strides3(0, st[0], st[1])
+
+
+def cp_pack_lse_rank(o: torch.Tensor, smax: torch.Tensor, ssum: torch.Tensor, W: int,
+                     scatter_dim: int = 1, pkt_o: Optional[torch.Tensor] = None,
+                     pkt_lse: Optional[torch.Tensor] = None,
+                     stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """This rank's send packet for W destinations: o [T, H, D], smax/ssum [T, H]
+    -> pkt_o [W, T, H/W, D], pkt_lse [W, T, H/W] (heads) or [W, T/W, H, D],
+    [W, T/W, H] (tokens); block j goes to destination j."""
+    _payload(o, "o", 3)
+    T, H, D = o.shape
+    _expect(smax, "smax", (T, H), torch.float32, o.device)
+    _expect(ssum, "ssum", (T, H), torch.float32, o.device)
+    shape = _packet_shape(W, T, H, scatter_dim)[1:]
+    shape = (W,) + shape
+    if pkt_o is None:
+        pkt_o = torch.empty(shape + (D,), dtype=o.dtype, device=o.device)
+    if pkt_lse is None:
+        pkt_lse = torch.empty(shape, dtype=torch.float32, device=o.device)
+    _expect(pkt_o, "pkt_o", shape + (D,), o.dtype, o.device)
+    _expect(pkt_lse, "pkt_lse", shape, torch.float32, o.device)
+    _dense(pkt_o, "pkt_o")
+    _dense(pkt_lse, "pkt_lse")
+    _check(_lib.cp_pack_lse_rank(_ptr(o), _strides_plane(o), _ptr(smax), _strides_plane(smax),
+                                 _ptr(ssum), _strides_plane(ssum), W, T, H, D, _dtype(o),
+                                 scatter_dim, _ptr(pkt_o), _ptr(pkt_lse), _stream(stream)))
+    return pkt_o, pkt_lse
+
+
+def cp_lse_combine_rank(recv_o: torch.Tensor, recv_lse: torch.Tensor,
+                        out: Optional[torch.Tensor] = None, out_lse: Optional[torch.Tensor] = None,
+                        stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One destination's combine: recv_o [W, T, Hc, D], recv_lse [W, T, Hc]
+    -> out [T, Hc, D], out_lse [T, Hc] (token chunks: T/W as T, H as Hc)."""
+    _payload(recv_o, "recv_o", 4)
+    W, T, Hc, D = recv_o.shape
+    _expect(recv_lse, "recv_lse", (W, T, Hc), torch.float32, recv_o.device)
+    if out is None:
+        out = torch.empty((T, Hc, D), dtype=recv_o.dtype, device=recv_o.device)
+    if out_lse is None:
+        out_lse = torch.empty((T, Hc), dtype=torch.float32, device=recv_o.device)
+    _expect(out, "out", (T, Hc, D), recv_o.dtype, recv_o.device)
+    _expect(out_lse, "out_lse", (T, Hc), torch.float32, recv_o.device)
+    for t, n in ((recv_o, "recv_o"), (recv_lse, "recv_lse"), (out, "out"), (out_lse, "out_lse")):
+        _dense(t, n)
+    _check(_lib.cp_lse_combine_rank(_ptr(recv_o), _ptr(recv_lse), W, T, Hc, D, _dtype(recv_o),
+                                    _ptr(out), _ptr(out_lse), _stream(stream)))
+    return out, out_lse
+
+
+def cp_pull_combine(o: Sequence, smax: Sequence, ssum: Sequence, dst: int, scatter_dim: int = 1,
+                    out: Optional[torch.Tensor] = None, out_lse: Optional[torch.Tensor] = None,
+                    device: Optional[torch.device] = None,
+                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Destination `dst` of W real ranks, pulled straight from every rank's
+    planes: o[r] [T, H, D], smax[r]/ssum[r] [T, H], all with the same strides.
+    A plane is a tensor of this device or any object with ``shape``, ``dtype``,
+    ``stride()`` and ``data_ptr()`` giving an address this device can read (a
+    peer's buffer mapped into this process). Returns out [T, H/W, D],
+    out_lse [T, H/W] (heads) or [T/W, H, D], [T/W, H] (tokens), on `device`
+    (default: the current device)."""
+    W = len(o)
+    if W < 1 or len(smax) != W or len(ssum) != W:
+        raise ValueError("o, smax and ssum must list the same W >= 1 ranks")
+    T, H, D = _plane(o[0], "o[0]", 3, None)
+    for r in range(W):
+        _plane(o[r], "o[%d]" % r, 3, o[0])
+        _plane(smax[r], "smax[%d]" % r, 2, smax[0], (T, H))
+        _plane(ssum[r], "ssum[%d]" % r, 2, ssum[0], (T, H))
+    if o[0].dtype not in (torch.bfloat16, torch.float16):
+        raise TypeError("payload dtype must be bfloat16 or float16, got %s" % o[0].dtype)
+    if smax[0].dtype != torch.float32 or ssum[0].dtype != torch.float32:
+        raise ValueError("smax and ssum must be float32")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    shape = _packet_shape(W, T, H, scatter_dim)[2:]
+    if out is None:
+        out = torch.empty(shape + (D,), dtype=o[0].dtype, device=dev)
+    if out_lse is None:
+        out_lse = torch.empty(shape, dtype=torch.float32, device=dev)
+    _expect(out, "out", shape + (D,), o[0].dtype, dev)
+    _expect(out_lse, "out_lse", shape, torch.float32, dev)
+    _dense(out, "out")
+    _dense(out_lse, "out_lse")
+    po = (ctypes.c_void_p * W)(*[t.data_ptr() for t in o])
+    pm = (ctypes.c_void_p * W)(*[t.data_ptr() for t in smax])
+    ps = (ctypes.c_void_p * W)(*[t.data_ptr() for t in ssum])
+    _check(_lib.cp_pull_combine(po, _strides_plane(o[0]), pm, _strides_plane(smax[0]), ps,
+                                _strides_plane(ssum[0]), W, T, H, D, _dtype(o[0]), scatter_dim,
+                                dst, _ptr(out), _ptr(out_lse), _stream(stream)))
+    return out, out_lse
+
+
+def _plane(t, name: str, ndim: int, like, shape=None):
+    """Shape (and, against `like`, dtype and strides) of one rank's plane."""
+    got = tuple(t.shape)
+    if len(got) != ndim:
+        raise ValueError("%s must have %d dimensions, got shape %s" % (name, ndim, got))
+    if shape is not None and got != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, got, tuple(shape)))
+    if like is not None:
+        if got != tuple(like.shape) or t.dtype != like.dtype:
+            raise ValueError("%s differs from the first rank's plane in shape or dtype" % name)
+        if tuple(t.stride()) != tuple(like.stride()):
+            raise ValueError("%s has other strides than the first rank's plane" % name)
+    return got
 
 
 def ulysses_seq2head(x: torch.Tensor, out: Optional[torch.Tensor] = None,

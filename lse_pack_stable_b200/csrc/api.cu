@@ -73,6 +73,38 @@ cp_status check_device_ptr(const void* p, const char* name)
     return CP_OK;
 }
 
+// The pointer must be device memory that the current device can address: its
+// own, or another device's (a peer mapping) when the two have peer access.
+cp_status check_addressable_ptr(const void* p, const char* name)
+{
+    if (p == nullptr) return fail(CP_ERR_ARG, "%s is NULL", name);
+    cudaPointerAttributes at;
+    cudaError_t e = cudaPointerGetAttributes(&at, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(CP_ERR_ARG, "%s: cudaPointerGetAttributes failed (%s)", name,
+                    cudaGetErrorString(e));
+    }
+    if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged)
+        return fail(CP_ERR_ARG, "%s is not device memory", name);
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(CP_ERR_CUDA, "cudaGetDevice failed");
+    }
+    if (at.type == cudaMemoryTypeDevice && at.device != dev) {
+        int can = 0;
+        if (cudaDeviceCanAccessPeer(&can, dev, at.device) != cudaSuccess) {
+            cudaGetLastError();
+            can = 0;
+        }
+        if (!can)
+            return fail(CP_ERR_ARG, "%s lives on device %d, which device %d cannot address", name,
+                        at.device, dev);
+    }
+    return CP_OK;
+}
+
 cp_status check_align(const void* p, int bytes, const char* name)
 {
     if (((uintptr_t)p) % (uintptr_t)bytes != 0)
@@ -181,6 +213,13 @@ cp_status check_devices(const void* const* p, const char* const* names, int n)
 
 }  // namespace
 
+// The message cp_last_error() returns, for the entry points in other files.
+cp_status cplse_set_error(cp_status st, const char* msg)
+{
+    snprintf(g_err, sizeof g_err, "%s", msg);
+    return st;
+}
+
 extern "C" {
 
 int cp_abi_version(void) { return CPLSE_ABI_VERSION; }
@@ -226,6 +265,7 @@ cp_status cp_pack_lse(const void* o, cp_strides3 so, const float* smax, cp_strid
     a.W = W; a.H = H; a.Hc = H / W; a.D = D; a.scatter_dim = scatter_dim;
     a.T = T; a.Tc = T / W;
     a.rows = rows;
+    a.nsrc = W;
     return launched(cplse::launch_pack(a, static_cast<cudaStream_t>(stream)), "cp_pack_lse");
 }
 
@@ -302,6 +342,7 @@ cp_status cp_pack_from_lse(const void* o, cp_strides3 so, const float* lse, cp_s
     a.W = W; a.H = H; a.Hc = H / W; a.D = D; a.scatter_dim = scatter_dim;
     a.T = T; a.Tc = T / W;
     a.rows = rows;
+    a.nsrc = W;
     return launched(cplse::launch_pack(a, static_cast<cudaStream_t>(stream)), "cp_pack_from_lse");
 }
 
@@ -415,6 +456,168 @@ cp_status cp_pack_permute_combine_fused(const void* o, cp_strides3 so, const flo
     return launched(cplse::launch_fused_async(a, static_cast<cplse::Dtype>(dt),
                                               static_cast<cudaStream_t>(stream)),
                     "cp_pack_permute_combine_fused");
+}
+
+cp_status cp_pack_lse_rank(const void* o, cp_strides3 so, const float* smax, cp_strides3 sm,
+                           const float* ssum, cp_strides3 ss, int W, int64_t T, int H, int D,
+                           cp_dtype dt, int scatter_dim, void* pkt_o, float* pkt_lse, void* stream)
+{
+    TRY(check_dims(W, T, H, D, dt));
+    if (scatter_dim != 0 && scatter_dim != 1)
+        return fail(CP_ERR_ARG, "scatter_dim must be 0 (tokens) or 1 (heads), got %d", scatter_dim);
+    if (scatter_dim == 0 && T % W != 0)
+        return fail(CP_ERR_SHAPE, "token scatter needs T %% W == 0 (T = %lld, W = %d)", (long long)T, W);
+    if (T == 0) return ok();
+    so.r = sm.r = ss.r = 0;                    // one source plane
+    TRY(check_sources(o, so, smax, sm, ssum, ss));
+    TRY(check_null(pkt_o, "pkt_o"));
+    TRY(check_null(pkt_lse, "pkt_lse"));
+    TRY(check_align(pkt_o, 16, "pkt_o"));
+    TRY(check_align(pkt_lse, 4, "pkt_lse"));
+    const int64_t rows = T * H;
+    const Span in[3] = {strided_span(o, 1, T, H, D, so, 2, "o"),
+                        strided_span(smax, 1, T, H, 1, sm, 4, "smax"),
+                        strided_span(ssum, 1, T, H, 1, ss, 4, "ssum")};
+    const Span out[2] = {dense_span(pkt_o, rows * D * 2, "pkt_o"),
+                         dense_span(pkt_lse, rows * 4, "pkt_lse")};
+    TRY(check_no_alias(in, 3, out, 2));
+    {
+        const void* p[5] = {o, smax, ssum, pkt_o, pkt_lse};
+        const char* n[5] = {"o", "smax", "ssum", "pkt_o", "pkt_lse"};
+        TRY(check_devices(p, n, 5));
+    }
+    cplse::PackArgs a{};
+    a.o = static_cast<const uint16_t*>(o);
+    a.so_r = 0; a.so_t = so.t; a.so_h = so.h;
+    a.smax = smax; a.ssum = ssum;
+    a.sm_r = 0; a.sm_t = sm.t; a.sm_h = sm.h;
+    a.ss_r = 0; a.ss_t = ss.t; a.ss_h = ss.h;
+    a.pkt_o = static_cast<uint16_t*>(pkt_o);
+    a.pkt_lse = pkt_lse;
+    a.W = W; a.H = H; a.Hc = H / W; a.D = D; a.scatter_dim = scatter_dim;
+    a.T = T; a.Tc = T / W;
+    a.rows = rows;
+    a.nsrc = 1;
+    return launched(cplse::launch_pack(a, static_cast<cudaStream_t>(stream)), "cp_pack_lse_rank");
+}
+
+cp_status cp_lse_combine_rank(const void* recv_o, const float* recv_lse, int W, int64_t T, int Hc,
+                              int D, cp_dtype dt, void* out, float* out_lse, void* stream)
+{
+    if (Hc < 1) return fail(CP_ERR_SHAPE, "Hc must be >= 1 (got %d)", Hc);
+    TRY(check_dims(W, T, Hc * W, D, dt));
+    if (T == 0) return ok();
+    TRY(check_null(recv_o, "recv_o"));
+    TRY(check_null(recv_lse, "recv_lse"));
+    TRY(check_null(out, "out"));
+    TRY(check_null(out_lse, "out_lse"));
+    TRY(check_align(recv_o, 16, "recv_o"));
+    TRY(check_align(recv_lse, 4, "recv_lse"));
+    TRY(check_align(out, 16, "out"));
+    TRY(check_align(out_lse, 4, "out_lse"));
+    const int64_t N = T * Hc;
+    const Span in[2] = {dense_span(recv_o, (int64_t)W * N * D * 2, "recv_o"),
+                        dense_span(recv_lse, (int64_t)W * N * 4, "recv_lse")};
+    const Span outs[2] = {dense_span(out, N * D * 2, "out"), dense_span(out_lse, N * 4, "out_lse")};
+    TRY(check_no_alias(in, 2, outs, 2));
+    {
+        const void* p[4] = {recv_o, recv_lse, out, out_lse};
+        const char* n[4] = {"recv_o", "recv_lse", "out", "out_lse"};
+        TRY(check_devices(p, n, 4));
+    }
+    // the received packet of one destination is destination 0 of a W-rank packet
+    cplse::CombineArgs a{};
+    a.src = static_cast<const uint16_t*>(recv_o);
+    a.rank_stride = N * D;
+    a.lse = recv_lse;
+    a.out = static_cast<uint16_t*>(out);
+    a.out_lse = out_lse;
+    a.W = W; a.H = Hc * W; a.Hc = Hc; a.D = D;
+    a.T = T; a.N = N; a.rows = N;
+    a.dense_rows = 1;
+    return launched(cplse::launch_combine_async(a, static_cast<cplse::Dtype>(dt),
+                                                static_cast<cudaStream_t>(stream)),
+                    "cp_lse_combine_rank");
+}
+
+cp_status cp_pull_combine(const void* const* o, cp_strides3 so, const float* const* smax,
+                          cp_strides3 sm, const float* const* ssum, cp_strides3 ss, int W,
+                          int64_t T, int H, int D, cp_dtype dt, int scatter_dim, int dst,
+                          void* out, float* out_lse, void* stream)
+{
+    TRY(check_dims(W, T, H, D, dt));
+    if (scatter_dim != 0 && scatter_dim != 1)
+        return fail(CP_ERR_ARG, "scatter_dim must be 0 (tokens) or 1 (heads), got %d", scatter_dim);
+    if (scatter_dim == 0 && T % W != 0)
+        return fail(CP_ERR_SHAPE, "token scatter needs T %% W == 0 (T = %lld, W = %d)", (long long)T, W);
+    if (dst < 0 || dst >= W) return fail(CP_ERR_ARG, "dst = %d is not a rank of 0..%d", dst, W - 1);
+    if (T == 0) return ok();
+    TRY(check_null(o, "o"));
+    TRY(check_null(smax, "smax"));
+    TRY(check_null(ssum, "ssum"));
+    so.r = sm.r = ss.r = 0;                    // every rank's plane has its own base
+    char nm[3][16];
+    for (int r = 0; r < W; ++r) {
+        snprintf(nm[0], sizeof nm[0], "o[%d]", r);
+        snprintf(nm[1], sizeof nm[1], "smax[%d]", r);
+        snprintf(nm[2], sizeof nm[2], "ssum[%d]", r);
+        TRY(check_null(o[r], nm[0]));
+        TRY(check_null(smax[r], nm[1]));
+        TRY(check_null(ssum[r], nm[2]));
+        TRY(check_align(o[r], 16, nm[0]));
+        TRY(check_align(smax[r], 4, nm[1]));
+        TRY(check_align(ssum[r], 4, nm[2]));
+    }
+    TRY(check_strides(so, true, "o"));
+    TRY(check_strides(sm, false, "smax"));
+    TRY(check_strides(ss, false, "ssum"));
+    TRY(check_null(out, "out"));
+    TRY(check_null(out_lse, "out_lse"));
+    TRY(check_align(out, 16, "out"));
+    TRY(check_align(out_lse, 4, "out_lse"));
+    const int Hc = H / W;
+    const int64_t Tc = T / W;
+    const int64_t rows = scatter_dim == 1 ? T * Hc : Tc * H;
+    const Span outs[2] = {dense_span(out, rows * D * 2, "out"),
+                          dense_span(out_lse, rows * 4, "out_lse")};
+    for (int r = 0; r < W; ++r) {
+        const Span in[3] = {strided_span(o[r], 1, T, H, D, so, 2, "o[r]"),
+                            strided_span(smax[r], 1, T, H, 1, sm, 4, "smax[r]"),
+                            strided_span(ssum[r], 1, T, H, 1, ss, 4, "ssum[r]")};
+        TRY(check_no_alias(in, 3, outs, 2));
+    }
+    {
+        const void* p[2] = {out, out_lse};
+        const char* n[2] = {"out", "out_lse"};
+        TRY(check_devices(p, n, 2));
+    }
+    for (int r = 0; r < W; ++r) {
+        snprintf(nm[0], sizeof nm[0], "o[%d]", r);
+        snprintf(nm[1], sizeof nm[1], "smax[%d]", r);
+        snprintf(nm[2], sizeof nm[2], "ssum[%d]", r);
+        TRY(check_addressable_ptr(o[r], nm[0]));
+        TRY(check_addressable_ptr(smax[r], nm[1]));
+        TRY(check_addressable_ptr(ssum[r], nm[2]));
+    }
+    cplse::PullArgs a{};
+    for (int r = 0; r < W; ++r) {
+        a.o[r] = static_cast<const uint16_t*>(o[r]);
+        a.smax[r] = smax[r];
+        a.ssum[r] = ssum[r];
+    }
+    a.so_t = so.t; a.so_h = so.h;
+    a.sm_t = sm.t; a.sm_h = sm.h;
+    a.ss_t = ss.t; a.ss_h = ss.h;
+    a.out = static_cast<uint16_t*>(out);
+    a.out_lse = out_lse;
+    a.W = W; a.H = H; a.Hc = Hc; a.D = D;
+    a.dst = dst;
+    a.token_scatter = scatter_dim == 0 ? 1 : 0;
+    a.T = T; a.Tc = Tc;
+    a.rows = rows;
+    return launched(cplse::launch_pull_combine(a, static_cast<cplse::Dtype>(dt),
+                                               static_cast<cudaStream_t>(stream)),
+                    "cp_pull_combine");
 }
 
 static cp_status ulysses(const void* in, void* out, int W, int B, int64_t S_local, int H, int D,

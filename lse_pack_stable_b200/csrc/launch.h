@@ -47,7 +47,25 @@ struct PackArgs {
     float* pkt_lse;
     int W, H, Hc, D, scatter_dim;
     int64_t T, Tc;
-    int64_t rows;             // W*T*H
+    int64_t rows;             // nsrc*T*H
+    int nsrc;                 // source ranks in this call: W (all simulated ranks) or 1 (one real rank)
+};
+
+// The pull-based exchange for one real destination rank: each source rank's
+// o/max/sum rows are read where they live (this GPU's memory or a peer's,
+// mapped into this process), through a table of per-rank base addresses.
+struct PullArgs {
+    const uint16_t* o[32];
+    const float* smax[32];
+    const float* ssum[32];
+    int64_t so_t, so_h, sm_t, sm_h, ss_t, ss_h;   // the same layout on every rank
+    uint16_t* out;
+    float* out_lse;
+    int W, H, Hc, D;
+    int dst;                  // this destination rank
+    int token_scatter;        // 0: head chunk dst (out [T][Hc][D]); 1: token chunk dst (out [T/W][H][D])
+    int64_t T, Tc;
+    int64_t rows;             // output rows
 };
 
 struct UlyssesArgs {
@@ -66,6 +84,7 @@ struct UlyssesArgs {
 cudaError_t launch_fused_async(const CombineArgs& a, Dtype dt, cudaStream_t s);
 cudaError_t launch_combine_async(const CombineArgs& a, Dtype dt, cudaStream_t s);
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t s);
+cudaError_t launch_pull_combine(const PullArgs& a, Dtype dt, cudaStream_t s);
 cudaError_t launch_lse_materialize(const PackArgs& a, float* lse, cudaStream_t s);
 cudaError_t launch_permute(const void* send, void* recv, int W, int64_t block_bytes,
                            cudaStream_t s);

@@ -152,7 +152,7 @@ template <bool FROM_LSE>
 __global__ void __launch_bounds__(kBlockThreads)
 pack_block_kernel(const PackArgs a, int64_t pay_cols)
 {
-    const int rj = blockIdx.y;
+    const int rj = blockIdx.y;                              // (source r, destination j)
     const int r = rj / a.W, j = rj - r * a.W;
     const int64_t HcV = (int64_t)a.Hc * (a.D >> 3);        // vectors per packet row
     const int64_t block_rows = a.T * a.Hc;
@@ -207,7 +207,7 @@ cudaError_t launch_pack_blocks(const PackArgs& a, cudaStream_t s)
     const int64_t pay_cols = (a.T * HcV + kBlockThreads * kBlockU - 1) / (kBlockThreads * kBlockU);
     const int64_t lse_cols = (a.T * a.Hc + kBlockThreads * 4 - 1) / (kBlockThreads * 4);
     if (pay_cols + lse_cols > 0x7fffffff) return cudaErrorInvalidConfiguration;
-    dim3 grid((unsigned)(pay_cols + lse_cols), (unsigned)(a.W * a.W));
+    dim3 grid((unsigned)(pay_cols + lse_cols), (unsigned)(a.nsrc * a.W));
     pack_block_kernel<FROM_LSE><<<grid, kBlockThreads, 0, s>>>(a, pay_cols);
     return cudaGetLastError();
 }

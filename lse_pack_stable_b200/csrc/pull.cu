@@ -1,0 +1,223 @@
+// Pull-based DCP exchange for one real destination rank: the fused
+// pack -> all-to-all -> combine across GPUs, in which destination j reads the
+// rows it combines straight out of every source rank's partial output and
+// statistics (peer memory over NVLink, mapped into this process) instead of
+// receiving a packet.
+//
+// Method: vLLM-Ascend pull request "Fuse local SFA LSE formation into DCP
+// pack", section "What this PR does / why we need it?": each source rank's
+// contribution to a row is LSE_r = softmax_max_r + log(softmax_sum_r), -inf
+// for invalid statistics; destination j, which owns head chunk j (or token
+// chunk j), merges the W contributions with the stable combine. The exchange
+// there is an HCCL all-to-all of the packed head chunks; here the destination
+// loads each source row once, with plain 16-byte global loads, so the packet
+// never exists on either side.
+//
+// Work split: the register-staged scheme of rowcombine.cuh. A warp owns chunks
+// of 32 output rows. Phase A: lane i forms the W LSE values of row i (one
+// coalesced float from each rank's max and sum plane) and the merge weights
+// (merge_weights, the arithmetic every merge kernel shares). Phase B: G lanes
+// cover a row with 16-byte vectors; every rank's vector of U steps is loaded
+// before any is used, accumulated in fp32 in rank order, rounded and stored.
+// A weight-0 contribution is neither loaded nor added (-0.0 stands in).
+//
+// No bulk copies, no TMA and no multicast: every remote byte arrives through
+// an ordinary load instruction, so nothing here depends on how the peer
+// memory was mapped beyond its being addressable from this device.
+#include <math.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "rowcombine.cuh"
+
+namespace cplse {
+namespace {
+
+constexpr int kPullThreads = 128;
+
+template <typename P, int WMAX, int G, int VPL, int U>
+__global__ void __launch_bounds__(kPullThreads) pull_combine_kernel(const PullArgs a)
+{
+    constexpr int RPI = 32 / G;          // rows per step
+    constexpr int STEPS = 32 / RPI;      // steps per chunk
+    constexpr int RB = WMAX < 16 ? WMAX : 16;   // ranks loaded at once
+    static_assert(STEPS % U == 0, "U must divide the steps of a chunk");
+
+    const int lane = threadIdx.x & 31;
+    const int sub = lane / G;
+    const int gl = lane % G;
+    const int64_t warp = ((int64_t)blockIdx.x * kPullThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * kPullThreads) >> 5;
+    const int64_t nchunks = (a.rows + 31) >> 5;
+    const int V = a.D >> 3;
+
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    for (int64_t c = warp; c < nchunks; c += nwarps) {
+        // ---------------- phase A: lane owns output row q
+        const int64_t q = c * 32 + lane;
+        const bool qv = q < a.rows;
+        int64_t t = 0, h = 0;
+        if (qv) {
+            if (a.token_scatter) {          // token chunk dst: row (tc, h), t = dst*Tc + tc
+                const int64_t tc = q / a.H;
+                h = q - tc * a.H;
+                t = (int64_t)a.dst * a.Tc + tc;
+            } else {                        // head chunk dst: row (t, hc), h = dst*Hc + hc
+                t = q / a.Hc;
+                h = (int64_t)a.dst * a.Hc + (q - t * a.Hc);
+            }
+        }
+        const int64_t src_row = t * a.so_t + h * a.so_h;
+        const int64_t mo = t * a.sm_t + h * a.sm_h;
+        const int64_t so = t * a.ss_t + h * a.ss_h;
+        float lse[WMAX];
+#pragma unroll
+        for (int r = 0; r < WMAX; ++r) {
+            float m = -INFINITY, sm = 0.f;
+            if (qv && r < a.W) {
+                m = ld_stream(a.smax[r] + mo);
+                sm = ld_stream(a.ssum[r] + so);
+            }
+            // invalid statistic: non-finite max, non-finite sum, or sum <= 0
+            const bool ok = isfinite(m) && isfinite(sm) && sm > 0.f;
+            lse[r] = ok ? m + logf(sm) : -INFINITY;
+        }
+        float w[WMAX];
+        float L;
+        const bool row_dead = !merge_weights(lse, w, L);
+        if (qv) st_stream(a.out_lse + q, L);
+
+        // ---------------- phase B: G lanes per row
+#pragma unroll 1
+        for (int s0 = 0; s0 < STEPS; s0 += U) {
+            int64_t sb[U];
+            bool rv[U], dead[U];
+            float ws[U][WMAX];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int k = (s0 + u) * RPI + sub;
+                sb[u] = __shfl_sync(kFull, src_row, k);
+                dead[u] = __shfl_sync(kFull, (int)row_dead, k) != 0;
+                rv[u] = c * 32 + k < a.rows;
+#pragma unroll
+                for (int r = 0; r < WMAX; ++r) ws[u][r] = __shfl_sync(kFull, w[r], k);
+            }
+            float acc[U][VPL][8];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int e = 0; e < VPL; ++e)
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) acc[u][e][x] = -0.f;
+
+#pragma unroll
+            for (int r0 = 0; r0 < WMAX; r0 += RB) {
+                uint4 v[U][VPL][RB];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+#pragma unroll
+                    for (int e = 0; e < VPL; ++e) {
+                        const int vec = gl + e * G;
+#pragma unroll
+                        for (int rr = 0; rr < RB; ++rr) {
+                            const int r = r0 + rr;
+                            if (rv[u] && vec < V && ws[u][r] != 0.f)
+                                v[u][e][rr] = ld_stream(
+                                    reinterpret_cast<const uint4*>(a.o[r] + sb[u]) + vec);
+                            else
+                                v[u][e][rr] = make_uint4(kNegZero2, kNegZero2, kNegZero2, kNegZero2);
+                        }
+                    }
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+#pragma unroll
+                    for (int e = 0; e < VPL; ++e)
+#pragma unroll
+                        for (int rr = 0; rr < RB; ++rr) {
+                            const float wr = ws[u][r0 + rr];
+                            const uint32_t wd[4] = {v[u][e][rr].x, v[u][e][rr].y, v[u][e][rr].z,
+                                                    v[u][e][rr].w};
+#pragma unroll
+                            for (int x = 0; x < 4; ++x) {
+                                const float2 f = unpack2<P>(wd[x]);
+                                acc[u][e][2 * x] = fmaf(wr, f.x, acc[u][e][2 * x]);
+                                acc[u][e][2 * x + 1] = fmaf(wr, f.y, acc[u][e][2 * x + 1]);
+                            }
+                        }
+            }
+
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int e = 0; e < VPL; ++e) {
+                    const int vec = gl + e * G;
+                    if (!(rv[u] && vec < V)) continue;
+                    uint4 o;
+                    if (dead[u]) {
+                        o = make_uint4(0u, 0u, 0u, 0u);   // all-invalid row: +0
+                    } else {
+                        o.x = pack2<P>(acc[u][e][0], acc[u][e][1]);
+                        o.y = pack2<P>(acc[u][e][2], acc[u][e][3]);
+                        o.z = pack2<P>(acc[u][e][4], acc[u][e][5]);
+                        o.w = pack2<P>(acc[u][e][6], acc[u][e][7]);
+                    }
+                    const int k = (s0 + u) * RPI + sub;
+                    st_stream(reinterpret_cast<uint4*>(a.out + (c * 32 + k) * a.D) + vec, o);
+                }
+        }
+    }
+}
+
+template <typename P, int WMAX, int G, int VPL>
+cudaError_t launch_pull_inst(const PullArgs& a, cudaStream_t s)
+{
+    constexpr int U0 = (WMAX * VPL) >= kLoadsInFlight ? 1 : kLoadsInFlight / (WMAX * VPL);
+    constexpr int U = U0 > G ? G : U0;
+    constexpr auto kern = pull_combine_kernel<P, WMAX, G, VPL, U>;
+    int per_sm = 0;
+    {
+        const cudaError_t e = resident_blocks<kern>(kPullThreads, 0, per_sm);
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t nchunks = (a.rows + 31) / 32;
+    int64_t blocks = (nchunks + kPullThreads / 32 - 1) / (kPullThreads / 32);
+    const int64_t cap = (int64_t)per_sm * sm_count();
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    return launch_pdl(kern, (unsigned)blocks, kPullThreads, 0, s, a);
+}
+
+template <typename P, int WMAX>
+cudaError_t launch_pull_w(const PullArgs& a, cudaStream_t s)
+{
+    const RowShape rs = row_shape(a.D);
+    switch (rs.G * 10 + rs.VPL) {
+    case 41: return launch_pull_inst<P, WMAX, 4, 1>(a, s);
+    case 81: return launch_pull_inst<P, WMAX, 8, 1>(a, s);
+    case 161: return launch_pull_inst<P, WMAX, 16, 1>(a, s);
+    case 321: return launch_pull_inst<P, WMAX, 32, 1>(a, s);
+    case 322: return launch_pull_inst<P, WMAX, 32, 2>(a, s);
+    default: return launch_pull_inst<P, WMAX, 32, 4>(a, s);
+    }
+}
+
+template <typename P>
+cudaError_t launch_pull_p(const PullArgs& a, cudaStream_t s)
+{
+    if (a.W <= 2) return launch_pull_w<P, 2>(a, s);
+    if (a.W <= 4) return launch_pull_w<P, 4>(a, s);
+    if (a.W <= 8) return launch_pull_w<P, 8>(a, s);
+    if (a.W <= 16) return launch_pull_w<P, 16>(a, s);
+    return launch_pull_w<P, 32>(a, s);
+}
+
+}  // namespace
+
+cudaError_t launch_pull_combine(const PullArgs& a, Dtype dt, cudaStream_t s)
+{
+    return dt == Dtype::kBf16 ? launch_pull_p<Bf16>(a, s) : launch_pull_p<Fp16>(a, s);
+}
+
+}  // namespace cplse

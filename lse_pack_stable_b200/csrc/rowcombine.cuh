@@ -46,6 +46,33 @@ constexpr uint32_t kNegZero2 = 0x80008000u;   // two -0.0 payload elements
 
 enum { kModeFused = 0, kModeCombine = 1 };
 
+// The merge weights of one row from its W contributions' LSE values (-inf for
+// an invalid contribution or one beyond W), in rank order: M = max_r lse_r;
+// if M = -inf the row is all invalid (returns false, every weight 0, L = -inf);
+// else L = M + logf(sum over valid r of expf(lse_r - M)) and
+// w_r = expf(lse_r - L) for valid r, 0 otherwise. Every merge kernel calls
+// this, so they all produce the same bits for the same LSE values.
+template <int WMAX, int NW>
+__device__ __forceinline__ bool merge_weights(const float (&lse)[WMAX], float (&w)[NW], float& L)
+{
+    static_assert(NW >= WMAX, "weight array shorter than the ranks");
+#pragma unroll
+    for (int r = 0; r < NW; ++r) w[r] = 0.f;
+    float M = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < WMAX; ++r) M = fmaxf(M, lse[r]);
+    L = -INFINITY;
+    if (!(M > -INFINITY)) return false;
+    float S = 0.f;
+#pragma unroll
+    for (int r = 0; r < WMAX; ++r)
+        if (lse[r] > -INFINITY) S += expf(lse[r] - M);
+    L = M + logf(S);
+#pragma unroll
+    for (int r = 0; r < WMAX; ++r) w[r] = lse[r] > -INFINITY ? expf(lse[r] - L) : 0.f;
+    return true;
+}
+
 // Phase A for one row: addresses and the W LSE values (-inf beyond W or q).
 template <int MODE, int WMAX>
 __device__ __forceinline__ void row_stats(const CombineArgs& a, int64_t q, bool qv,
@@ -130,26 +157,10 @@ rowcombine_kernel(const CombineArgs a)
         float lse[WMAX];
         row_stats<MODE, WMAX>(a, q, qv, src_row, dst_row, lse);
 
-        float M = -INFINITY;
-#pragma unroll
-        for (int r = 0; r < WMAX; ++r) M = fmaxf(M, lse[r]);
         float w[WMAX];
-        float L = -INFINITY;
-        if (M > -INFINITY) {
-            float S = 0.f;
-#pragma unroll
-            for (int r = 0; r < WMAX; ++r)
-                if (lse[r] > -INFINITY) S += expf(lse[r] - M);
-            L = M + logf(S);
-#pragma unroll
-            for (int r = 0; r < WMAX; ++r)
-                w[r] = lse[r] > -INFINITY ? expf(lse[r] - L) : 0.f;
-        } else {
-#pragma unroll
-            for (int r = 0; r < WMAX; ++r) w[r] = 0.f;
-        }
+        float L;
+        const bool row_dead = !merge_weights(lse, w, L);
         if (qv) st_stream(a.out_lse + dst_row, L);
-        const bool row_dead = !(M > -INFINITY);
 
         // ---------------- phase B: G lanes per row
 #pragma unroll 1
@@ -236,9 +247,9 @@ rowcombine_kernel(const CombineArgs a)
 // the next grid's scheduling with this one's drain. Every merge kernel opens
 // with griddepcontrol.wait, so none reads memory before the previous kernel in
 // the stream has completed.
-template <typename K>
+template <typename K, typename A>
 cudaError_t launch_pdl(K kern, unsigned blocks, int threads, int smem, cudaStream_t s,
-                       const CombineArgs& a)
+                       const A& a)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(blocks);

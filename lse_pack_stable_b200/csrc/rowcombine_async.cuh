@@ -247,29 +247,16 @@ rowcombine_async_kernel(const CombineArgs a)
                     lse[r] = x > -INFINITY ? x : -INFINITY;
                 }
             }
-            float M = -INFINITY;
-#pragma unroll
-            for (int r = 0; r < WMAX; ++r) M = fmaxf(M, lse[r]);
-            float L = -INFINITY;
+            float L;
             float w[WS];
-#pragma unroll
-            for (int r = 0; r < WS; ++r) w[r] = 0.f;
-            if (M > -INFINITY) {
-                float S = 0.f;
-#pragma unroll
-                for (int r = 0; r < WMAX; ++r)
-                    if (lse[r] > -INFINITY) S += expf(lse[r] - M);
-                L = M + logf(S);
-#pragma unroll
-                for (int r = 0; r < WMAX; ++r) w[r] = lse[r] > -INFINITY ? expf(lse[r] - L) : 0.f;
-            }
+            const bool alive = merge_weights(lse, w, L);
             if (qv) st_stream(a.out_lse + dst, L);
             __syncwarp();                                   // the previous chunk's table is read
 #pragma unroll
             for (int r = 0; r < WS; r += 4)
                 *reinterpret_cast<float4*>(wtab + lane * WS + r) =
                     make_float4(w[r], w[r + 1], w[r + 2], w[r + 3]);
-            dtab[lane] = (M > -INFINITY) ? dst : ~dst;
+            dtab[lane] = alive ? dst : ~dst;
             __syncwarp();                                   // the table is visible to the warp
         }
         // ---------------- phase B: this step's RPI rows, G lanes per row

@@ -41,7 +41,7 @@ def test_only_declared_symbols_are_exported():
 
 
 def test_abi_version():
-    assert cp.abi_version() == cp.ABI_VERSION == 2
+    assert cp.abi_version() == cp.ABI_VERSION == 3
 
 
 # aligned fake addresses: host checks run before any pointer is dereferenced or queried
@@ -174,3 +174,92 @@ def test_binding_rejects_noncontiguous_and_dtype():
         cp.cp_pack_permute_combine_fused(ob, torch.zeros(2, 4, 8), torch.zeros(2, 4, 8),
                                          out=torch.zeros(2, 4, 4, 64, dtype=torch.bfloat16),
                                          out_lse=torch.zeros(2, 4, 4))
+
+
+# ---- the per-rank entry points of the exchange across real ranks
+
+
+def _pack_rank(W=2, T=4, H=8, D=64, dt=0, sd=1, o=A, m=2 * A, s=3 * A, po=4 * A, pl=5 * A):
+    return L.cp_pack_lse_rank(o, S(0, H * D, D), m, S(0, H, 1), s, S(0, H, 1), W, T, H, D, dt,
+                              sd, po, pl, None)
+
+
+@pytest.mark.parametrize("kw,status,msg", [
+    (dict(W=3), cp.CP_ERR_SHAPE, "multiple of W"),
+    (dict(sd=0, T=5), cp.CP_ERR_SHAPE, "T % W"),
+    (dict(o=0), cp.CP_ERR_ARG, "o is NULL"),
+    (dict(po=4 * A + 8), cp.CP_ERR_ALIGN, "pkt_o is not 16-byte aligned"),
+    # one plane: T*H*D*2 = 4 KiB of o; the packet starting inside it overlaps
+    (dict(po=A + 4096 - 16), cp.CP_ERR_ALIAS, "pkt_o overlaps input o"),
+])
+def test_pack_rank_rejects(kw, status, msg):
+    assert _pack_rank(**kw) == status
+    assert msg in cp.last_error()
+
+
+def test_pack_rank_one_plane_spans():
+    # a packet right after one plane (T*H*D*2 bytes) does not overlap it: only
+    # one source plane is read, whatever W is
+    assert _pack_rank(po=A + 4096) == cp.CP_ERR_ARG and _device_check_failed("o")
+    assert _pack_rank(T=0, o=0, m=0, s=0, po=0, pl=0) == cp.CP_OK
+
+
+@pytest.mark.parametrize("args,status,msg", [
+    ((A, 2 * A, 2, 4, 0, 64, 0, 4 * A, 5 * A), cp.CP_ERR_SHAPE, "Hc must be"),
+    ((A, 2 * A, 2, 4, 4, 64, 0, A + 16, 5 * A), cp.CP_ERR_ALIAS, "out overlaps input recv_o"),
+    ((A, 2 * A, 2, 4, 4, 64, 0, 4 * A + 2, 5 * A), cp.CP_ERR_ALIGN, "out is not 16"),
+])
+def test_combine_rank_rejects(args, status, msg):
+    assert L.cp_lse_combine_rank(*args, None) == status
+    assert msg in cp.last_error()
+
+
+def _table(*addrs):
+    return (ctypes.c_void_p * len(addrs))(*addrs)
+
+
+def _pull(W=2, T=4, H=8, D=64, dt=0, sd=1, dst=0, o=None, m=None, s=None, out=8 * A,
+          ol=9 * A):
+    o = o if o is not None else _table(*[A + r * (A // 4) for r in range(W)])
+    m = m if m is not None else _table(*[2 * A + r * (A // 4) for r in range(W)])
+    s = s if s is not None else _table(*[3 * A + r * (A // 4) for r in range(W)])
+    return L.cp_pull_combine(o, S(0, H * D, D), m, S(0, H, 1), s, S(0, H, 1), W, T, H, D, dt, sd,
+                             dst, out, ol, None)
+
+
+@pytest.mark.parametrize("kw,status,msg", [
+    (dict(dst=2), cp.CP_ERR_ARG, "dst = 2"),
+    (dict(dst=-1), cp.CP_ERR_ARG, "dst = -1"),
+    (dict(W=3), cp.CP_ERR_SHAPE, "multiple of W"),
+    (dict(sd=0, T=5), cp.CP_ERR_SHAPE, "T % W"),
+    (dict(o=_table(A, 0)), cp.CP_ERR_ARG, "o[1] is NULL"),
+    (dict(s=_table(3 * A, 3 * A + 2)), cp.CP_ERR_ALIGN, "ssum[1] is not 4-byte aligned"),
+    (dict(o=_table(A + 8, A + A // 4)), cp.CP_ERR_ALIGN, "o[0] is not 16-byte aligned"),
+    (dict(out=A + A // 4 + 64), cp.CP_ERR_ALIAS, "out overlaps input o[r]"),
+    (dict(ol=0), cp.CP_ERR_ARG, "out_lse is NULL"),
+])
+def test_pull_rejects(kw, status, msg):
+    assert _pull(**kw) == status
+    assert msg in cp.last_error()
+
+
+def test_pull_null_tables_and_device_check():
+    assert L.cp_pull_combine(None, S(0, 512, 64), None, S(0, 8, 1), None, S(0, 8, 1), 2, 4, 8,
+                             64, 0, 1, 0, 8 * A, 9 * A, None) == cp.CP_ERR_ARG
+    assert "o is NULL" in cp.last_error()
+    # every host check passes; the driver check then refuses the fake addresses
+    assert _pull() == cp.CP_ERR_ARG and _device_check_failed("out")
+
+
+def test_ipc_calls_reject_bad_arguments():
+    h = cp.IpcHandle()
+    assert L.cp_ipc_export(None, ctypes.byref(h)) == cp.CP_ERR_ARG and "p is NULL" in cp.last_error()
+    assert L.cp_ipc_export(A, None) == cp.CP_ERR_ARG and "h is NULL" in cp.last_error()
+    # a host address: the driver query refuses it (no GPU here, or not device memory)
+    assert L.cp_ipc_export(A, ctypes.byref(h)) == cp.CP_ERR_ARG
+    base, p = ctypes.c_void_p(), ctypes.c_void_p()
+    h.offset, h.alloc_bytes = 64, 64
+    assert L.cp_ipc_import(ctypes.byref(h), ctypes.byref(base), ctypes.byref(p)) == cp.CP_ERR_ARG
+    assert "outside" in cp.last_error()
+    assert L.cp_ipc_import(None, ctypes.byref(base), ctypes.byref(p)) == cp.CP_ERR_ARG
+    assert L.cp_ipc_close(None) == cp.CP_ERR_ARG
