@@ -67,6 +67,9 @@ def parse(argv=None):
                          "(one GPU only); 'none' for the headline alone")
     ap.add_argument("--launches", type=int, default=ROOFLINE_LAUNCHES,
                     help="event-bracketed launches of the roofline pass (at least 50)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="cut the headline workload to this many tokens (small cases for "
+                         "profiler captures; 0: the workload's own T)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -584,6 +587,8 @@ def run_ours(args):
         pass
 
     wl = synth.CONFIGS[args.config]
+    if args.tokens > 0:
+        wl = synth.Workload(**{**wl.__dict__, "T": args.tokens})
     stream = torch.cuda.current_stream(dev)
 
     head = measure_workload(cp, wl, dev, stream, args, 1, barrier, peak, peak_kind, True)

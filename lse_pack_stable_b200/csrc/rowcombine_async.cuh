@@ -38,6 +38,11 @@ namespace cplse {
 #ifndef CPLSE_ASYNC_INFLIGHT
 #define CPLSE_ASYNC_INFLIGHT 4096
 #endif
+#ifndef CPLSE_ASYNC_L2AHEAD
+#define CPLSE_ASYNC_L2AHEAD 0
+#endif
+// steps beyond the ring whose payload each warp asks the L2 to fetch early
+constexpr int kL2Ahead = CPLSE_ASYNC_L2AHEAD;
 constexpr int kAsyncThreads = CPLSE_ASYNC_THREADS;
 // payload bytes each warp keeps in flight (sets the ring depth NST)
 constexpr int kAsyncInflight = CPLSE_ASYNC_INFLIGHT;
@@ -55,6 +60,11 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src)
 __device__ __forceinline__ void cp_async_f32(uint32_t dst, const void* src)
 {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void prefetch_l2_line(const void* p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 __device__ __forceinline__ void cp_async_commit()
@@ -180,6 +190,26 @@ rowcombine_async_kernel(const CombineArgs a)
             }
             const int64_t q = c * 32 + st_i * RPI + sub;
             if (st_i == 0) chunk_src = row_src(c * 32);   // rank-0 offset of the chunk's row 0
+            if (kL2Ahead > 0 && linear_chunks) {
+                // L2 prefetch of later steps of this chunk: step st_i + kL2Ahead, and
+                // on the chunk's first group the steps the ring's prologue skips
+                auto pf = [&](int sp) {
+                    const int64_t qp = c * 32 + sp * RPI + sub;
+                    if (sp < STEPS && qp < a.rows) {
+                        const uint4* bp = src16 + chunk_src + (sp * RPI + sub) * V + gl;
+#pragma unroll
+                        for (int e = 0; e < VPL; ++e)
+                            if (gl + e * G < V) {
+#pragma unroll
+                                for (int r = 0; r < WMAX; ++r)
+                                    if (r < W) prefetch_l2_line(bp + e * G + r * rs16);
+                            }
+                    }
+                };
+                if (st_i == 0)
+                    for (int sp = NST - 1; sp < kL2Ahead; ++sp) pf(sp);
+                pf(st_i + kL2Ahead);
+            }
             if (q < a.rows) {
                 // rows of a chunk are consecutive rows of one block when the block
                 // row count is a multiple of 32 (combine) or rows are dense (fused)
