@@ -328,8 +328,7 @@ def cp_pack_lse_rank(o: torch.Tensor, smax: torch.Tensor, ssum: torch.Tensor, W:
     T, H, D = o.shape
     _expect(smax, "smax", (T, H), torch.float32, o.device)
     _expect(ssum, "ssum", (T, H), torch.float32, o.device)
-    shape = _packet_shape(W, T, H, scatter_dim)[1:]
-    shape = (W,) + shape
+    shape = _packet_shape(W, T, H, scatter_dim)[1:]        # [W_dst, rows...]
     if pkt_o is None:
         pkt_o = torch.empty(shape + (D,), dtype=o.dtype, device=o.device)
     if pkt_lse is None:

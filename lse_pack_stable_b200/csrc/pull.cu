@@ -48,16 +48,20 @@ __global__ void __launch_bounds__(kPullThreads) pull_combine_kernel(const PullAr
     const int gl = lane % G;
     const int64_t warp = ((int64_t)blockIdx.x * kPullThreads + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * kPullThreads) >> 5;
-    const int64_t nchunks = (a.rows + 31) >> 5;
+    const ChunkPlan plan(a.rows, warp, nwarps);
     const int V = a.D >> 3;
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    for (int64_t c = warp; c < nchunks; c += nwarps) {
-        // ---------------- phase A: lane owns output row q
-        const int64_t q = c * 32 + lane;
-        const bool qv = q < a.rows;
+    const int64_t my_chunks = plan.count();
+    for (int64_t ci = 0; ci < my_chunks; ++ci) {
+        int64_t c0;
+        int cn;
+        plan.chunk(ci, c0, cn);
+        // ---------------- phase A: lane owns output row q = c0 + lane
+        const int64_t q = c0 + lane;
+        const bool qv = lane < cn;
         int64_t t = 0, h = 0;
         if (qv) {
             if (a.token_scatter) {          // token chunk dst: row (tc, h), t = dst*Tc + tc
@@ -100,7 +104,7 @@ __global__ void __launch_bounds__(kPullThreads) pull_combine_kernel(const PullAr
                 const int k = (s0 + u) * RPI + sub;
                 sb[u] = __shfl_sync(kFull, src_row, k);
                 dead[u] = __shfl_sync(kFull, (int)row_dead, k) != 0;
-                rv[u] = c * 32 + k < a.rows;
+                rv[u] = k < cn;
 #pragma unroll
                 for (int r = 0; r < WMAX; ++r) ws[u][r] = __shfl_sync(kFull, w[r], k);
             }
@@ -164,7 +168,7 @@ __global__ void __launch_bounds__(kPullThreads) pull_combine_kernel(const PullAr
                         o.w = pack2<P>(acc[u][e][6], acc[u][e][7]);
                     }
                     const int k = (s0 + u) * RPI + sub;
-                    st_stream(reinterpret_cast<uint4*>(a.out + (c * 32 + k) * a.D) + vec, o);
+                    st_stream(reinterpret_cast<uint4*>(a.out + (c0 + k) * a.D) + vec, o);
                 }
         }
     }

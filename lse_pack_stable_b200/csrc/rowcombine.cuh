@@ -46,6 +46,47 @@ constexpr uint32_t kNegZero2 = 0x80008000u;   // two -0.0 payload elements
 
 enum { kModeFused = 0, kModeCombine = 1 };
 
+// How a grid's warps share the output rows of a merge. Full rounds first: in
+// round k, warp w takes the 32-row chunk k*nwarps + w, so that warps working
+// at the same time read neighbouring rows. The rows left after the last full
+// round (fewer than 32 per warp) are then split evenly, ceil(rem / nwarps) per
+// warp, rather than as whole chunks to some warps only: a whole chunk can be
+// hundreds of KB of payload, and the warps that would take an extra one would
+// keep the grid running long after the others had finished.
+struct ChunkPlan {
+    int64_t rows, warp, nwarps;
+    int64_t full;             // full rounds of 32-row chunks
+    int64_t last_base;        // first row of the last, partial round
+    int64_t last_rows;        // rows per warp in the last round (<= 32)
+
+    __device__ __forceinline__ ChunkPlan(int64_t rows_, int64_t warp_, int64_t nwarps_)
+        : rows(rows_), warp(warp_), nwarps(nwarps_)
+    {
+        full = rows / (32 * nwarps);
+        last_base = full * 32 * nwarps;
+        last_rows = (rows - last_base + nwarps - 1) / nwarps;
+    }
+
+    // chunks of this warp
+    __device__ __forceinline__ int64_t count() const
+    {
+        return full + (last_base + warp * last_rows < rows ? 1 : 0);
+    }
+
+    // chunk i of this warp: its first row and its row count (1..32)
+    __device__ __forceinline__ void chunk(int64_t i, int64_t& start, int& n) const
+    {
+        if (i < full) {
+            start = (warp + i * nwarps) * 32;
+            n = 32;
+        } else {
+            start = last_base + warp * last_rows;
+            const int64_t left = rows - start;
+            n = (int)(left < last_rows ? left : last_rows);
+        }
+    }
+};
+
 // The merge weights of one row from its W contributions' LSE values (-inf for
 // an invalid contribution or one beyond W), in rank order: M = max_r lse_r;
 // if M = -inf the row is all invalid (returns false, every weight 0, L = -inf);
@@ -138,7 +179,7 @@ rowcombine_kernel(const CombineArgs a)
     const int gl = lane % G;
     const int64_t warp = ((int64_t)blockIdx.x * kCombineThreads + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * kCombineThreads) >> 5;
-    const int64_t nchunks = (a.rows + 31) >> 5;
+    const ChunkPlan plan(a.rows, warp, nwarps);
     const int V = a.D >> 3;
     const int64_t rank_stride = a.rank_stride;
 
@@ -149,10 +190,14 @@ rowcombine_kernel(const CombineArgs a)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    for (int64_t c = warp; c < nchunks; c += nwarps) {
-        // ---------------- phase A: lane owns row c*32 + lane
-        const int64_t q = c * 32 + lane;
-        const bool qv = q < a.rows;
+    const int64_t my_chunks = plan.count();
+    for (int64_t ci = 0; ci < my_chunks; ++ci) {
+        int64_t c0;
+        int cn;
+        plan.chunk(ci, c0, cn);
+        // ---------------- phase A: lane owns row c0 + lane
+        const int64_t q = c0 + lane;
+        const bool qv = lane < cn;
         int64_t src_row, dst_row;
         float lse[WMAX];
         row_stats<MODE, WMAX>(a, q, qv, src_row, dst_row, lse);
@@ -174,7 +219,7 @@ rowcombine_kernel(const CombineArgs a)
                 sb[u] = __shfl_sync(kFull, src_row, k);
                 db[u] = __shfl_sync(kFull, dst_row, k);
                 dead[u] = __shfl_sync(kFull, (int)row_dead, k) != 0;
-                rv[u] = c * 32 + k < a.rows;
+                rv[u] = k < cn;
 #pragma unroll
                 for (int r = 0; r < WMAX; ++r) ws[u][r] = __shfl_sync(kFull, w[r], k);
             }

@@ -131,9 +131,8 @@ rowcombine_async_kernel(const CombineArgs a)
     const uint4* src16 = reinterpret_cast<const uint4*>(a.src);
     const int64_t warp = ((int64_t)blockIdx.x * kAsyncThreads + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * kAsyncThreads) >> 5;
-    const int64_t nchunks = (a.rows + 31) >> 5;
-    const int64_t my_chunks = warp < nchunks ? (nchunks - warp + nwarps - 1) / nwarps : 0;
-    const int64_t ngroups = my_chunks * STEPS;
+    const ChunkPlan plan(a.rows, warp, nwarps);
+    const int64_t ngroups = plan.count() * STEPS;
 
     // Programmatic dependent launch: the next kernel in the stream may be
     // scheduled now, and this one reads nothing until the previous kernel in
@@ -155,17 +154,28 @@ rowcombine_async_kernel(const CombineArgs a)
         }
     };
 
-    const bool linear_chunks = MODE == kModeFused ? a.dense_rows != 0 : (a.N & 31) == 0;
+    // A chunk's rows are consecutive rows of one source block -- so that their
+    // payload offsets are those of its first row plus k*D -- when rows are
+    // dense (fused), or when the chunk stays inside one (dst) block (combine).
+    auto chunk_is_linear = [&](int64_t c0, int cn) -> bool {
+        if (MODE == kModeFused) return a.dense_rows != 0;
+        return c0 / a.N == (c0 + cn - 1) / a.N;
+    };
 
     // issue cursor: group ni = chunk ci_i, step st_i, ring slot sl_i
-    int64_t ni = 0, ci_i = 0, chunk_src = 0;
-    int st_i = 0, sl_i = 0;
+    int64_t ni = 0, ci_i = 0, chunk_src = 0, c0_i = 0;
+    int st_i = 0, sl_i = 0, cn_i = 0;
+    bool lin_i = false;
     auto issue_next = [&]() {
         if (ni < ngroups) {
-            const int64_t c = warp + ci_i * nwarps;
+            if (st_i == 0) {
+                plan.chunk(ci_i, c0_i, cn_i);
+                lin_i = chunk_is_linear(c0_i, cn_i);
+                chunk_src = row_src(c0_i);                 // rank-0 offset of the chunk's row 0
+            }
             if (st_i == 0) {   // this chunk's statistics, lane = row
-                const int64_t q = c * 32 + lane;
-                if (q < a.rows) {
+                const int64_t q = c0_i + lane;
+                if (lane < cn_i) {
                     float* sl = sring + (int)(ci_i % Ring::kStat) * Ring::kStatSlotFloats;
                     if (MODE == kModeFused) {
                         int64_t t, h;
@@ -188,14 +198,12 @@ rowcombine_async_kernel(const CombineArgs a)
                     }
                 }
             }
-            const int64_t q = c * 32 + st_i * RPI + sub;
-            if (st_i == 0) chunk_src = row_src(c * 32);   // rank-0 offset of the chunk's row 0
-            if (kL2Ahead > 0 && linear_chunks) {
+            const int kq = st_i * RPI + sub;                 // row of the chunk
+            if (kL2Ahead > 0 && lin_i) {
                 // L2 prefetch of later steps of this chunk: step st_i + kL2Ahead, and
                 // on the chunk's first group the steps the ring's prologue skips
                 auto pf = [&](int sp) {
-                    const int64_t qp = c * 32 + sp * RPI + sub;
-                    if (sp < STEPS && qp < a.rows) {
+                    if (sp < STEPS && sp * RPI + sub < cn_i) {
                         const uint4* bp = src16 + chunk_src + (sp * RPI + sub) * V + gl;
 #pragma unroll
                         for (int e = 0; e < VPL; ++e)
@@ -210,10 +218,8 @@ rowcombine_async_kernel(const CombineArgs a)
                     for (int sp = NST - 1; sp < kL2Ahead; ++sp) pf(sp);
                 pf(st_i + kL2Ahead);
             }
-            if (q < a.rows) {
-                // rows of a chunk are consecutive rows of one block when the block
-                // row count is a multiple of 32 (combine) or rows are dense (fused)
-                const int64_t off = linear_chunks ? chunk_src + (st_i * RPI + sub) * V : row_src(q);
+            if (kq < cn_i) {
+                const int64_t off = lin_i ? chunk_src + kq * V : row_src(c0_i + kq);
                 const uint4* base = src16 + off + gl;
                 uint4* sl = ring + sl_i * Ring::kSlotVecs + lane;
 #pragma unroll
@@ -239,16 +245,16 @@ rowcombine_async_kernel(const CombineArgs a)
 #pragma unroll 1
     for (int d = 0; d < NST - 1; ++d) issue_next();
 
-    int64_t ci = 0;
-    int step = 0, slot = 0;
+    int64_t ci = 0, c0 = 0;
+    int step = 0, slot = 0, cn = 0;
     for (int64_t n = 0; n < ngroups; ++n) {
         cp_async_wait<NST - 2>();       // group n has landed (this lane's copies)
         issue_next();                   // refill the slot that group n-1 used
-        const int64_t c = warp + ci * nwarps;
+        if (step == 0) plan.chunk(ci, c0, cn);
         if (step == 0) {
-            // ---------------- phase A: lane owns row c*32 + lane
-            const int64_t q = c * 32 + lane;
-            const bool qv = q < a.rows;
+            // ---------------- phase A: lane owns row c0 + lane
+            const int64_t q = c0 + lane;
+            const bool qv = lane < cn;
             int64_t dst = 0;
             if (qv) {
                 if (MODE == kModeFused && !a.token_scatter) {
@@ -291,8 +297,7 @@ rowcombine_async_kernel(const CombineArgs a)
         }
         // ---------------- phase B: this step's RPI rows, G lanes per row
         const int k = step * RPI + sub;                     // row of the chunk
-        const int64_t q = c * 32 + k;
-        if (q < a.rows) {
+        if (k < cn) {
             int64_t db = dtab[k];
             const bool dead = db < 0;
             if (dead) db = ~db;
