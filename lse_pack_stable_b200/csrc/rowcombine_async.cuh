@@ -38,11 +38,7 @@ namespace cplse {
 #ifndef CPLSE_ASYNC_INFLIGHT
 #define CPLSE_ASYNC_INFLIGHT 4096
 #endif
-#ifndef CPLSE_ASYNC_L2AHEAD
-#define CPLSE_ASYNC_L2AHEAD 0
-#endif
-// steps beyond the ring whose payload each warp asks the L2 to fetch early
-constexpr int kL2Ahead = CPLSE_ASYNC_L2AHEAD;
+
 constexpr int kAsyncThreads = CPLSE_ASYNC_THREADS;
 // payload bytes each warp keeps in flight (sets the ring depth NST)
 constexpr int kAsyncInflight = CPLSE_ASYNC_INFLIGHT;
@@ -60,11 +56,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src)
 __device__ __forceinline__ void cp_async_f32(uint32_t dst, const void* src)
 {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-
-__device__ __forceinline__ void prefetch_l2_line(const void* p)
-{
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 __device__ __forceinline__ void cp_async_commit()
@@ -199,25 +190,6 @@ rowcombine_async_kernel(const CombineArgs a)
                 }
             }
             const int kq = st_i * RPI + sub;                 // row of the chunk
-            if (kL2Ahead > 0 && lin_i) {
-                // L2 prefetch of later steps of this chunk: step st_i + kL2Ahead, and
-                // on the chunk's first group the steps the ring's prologue skips
-                auto pf = [&](int sp) {
-                    if (sp < STEPS && sp * RPI + sub < cn_i) {
-                        const uint4* bp = src16 + chunk_src + (sp * RPI + sub) * V + gl;
-#pragma unroll
-                        for (int e = 0; e < VPL; ++e)
-                            if (gl + e * G < V) {
-#pragma unroll
-                                for (int r = 0; r < WMAX; ++r)
-                                    if (r < W) prefetch_l2_line(bp + e * G + r * rs16);
-                            }
-                    }
-                };
-                if (st_i == 0)
-                    for (int sp = NST - 1; sp < kL2Ahead; ++sp) pf(sp);
-                pf(st_i + kL2Ahead);
-            }
             if (kq < cn_i) {
                 const int64_t off = lin_i ? chunk_src + kq * V : row_src(c0_i + kq);
                 const uint4* base = src16 + off + gl;
