@@ -55,7 +55,7 @@ extern "C" {
 #define CPLSE_API
 #endif
 
-#define CPLSE_ABI_VERSION 3
+#define CPLSE_ABI_VERSION 4
 #define CPLSE_MAX_W 32     /* simulated ranks per call */
 #define CPLSE_MAX_D 1024   /* head dim, elements */
 
@@ -281,6 +281,29 @@ CPLSE_API cp_status ulysses_seq2head(const void* in, void* out, int W, int B, in
  */
 CPLSE_API cp_status ulysses_head2seq(const void* in, void* out, int W, int B, int64_t S_local, int H, int D,
                            int elem_bytes, void* stream);
+
+/*
+ * [ULY] The Ulysses all-to-alls across W real ranks, one per GPU, as a
+ * load/store exchange over NVLink: destination `dst` reads its share of every
+ * rank's tensor where it lives and writes its own result, byte-identical to
+ * the NCCL all_to_all_4D and to block dst of the single-GPU calls above.
+ *   in   HOST array of W device addresses: rank r's tensor (this device's
+ *        memory, or a peer's mapped into this process with cp_ipc_import)
+ *   out  destination dst's tensor, on the current device
+ * seq2head: in[r] [B][S_local][H][D] -> out [B][W*S_local][H/W][D],
+ *           out[b][r*S_local + s][hc] = in[r][b][s][dst*Hc + hc]
+ * head2seq: in[r] [B][W*S_local][H/W][D] -> out [B][S_local][H][D],
+ *           out[b][s][r*Hc + hc] = in[r][b][dst*S_local + s][hc]
+ * Ordinary loads and stores only (no bulk or multicast copies); the caller
+ * orders the call after every rank's writes to its tensor and before any
+ * rank overwrites it again. B <= 65535.
+ */
+CPLSE_API cp_status ulysses_seq2head_pull(const void* const* in, void* out, int W, int B,
+                                          int64_t S_local, int H, int D, int elem_bytes, int dst,
+                                          void* stream);
+CPLSE_API cp_status ulysses_head2seq_pull(const void* const* in, void* out, int W, int B,
+                                          int64_t S_local, int H, int D, int elem_bytes, int dst,
+                                          void* stream);
 
 #ifdef __cplusplus
 }

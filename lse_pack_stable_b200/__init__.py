@@ -41,7 +41,8 @@ EXPORTS = ("cp_abi_version", "cp_last_error", "cp_pack_lse", "cp_lse_materialize
            "cp_pack_from_lse", "cp_a2a_local_permute",
            "cp_lse_combine", "cp_pack_permute_combine_fused", "cp_pack_lse_rank",
            "cp_lse_combine_rank", "cp_pull_combine", "cp_ipc_export", "cp_ipc_import",
-           "cp_ipc_close", "ulysses_seq2head", "ulysses_head2seq")
+           "cp_ipc_close", "ulysses_seq2head", "ulysses_head2seq", "ulysses_seq2head_pull",
+           "ulysses_head2seq_pull")
 
 
 class Strides3(ctypes.Structure):
@@ -51,7 +52,7 @@ class Strides3(ctypes.Structure):
 _p, _i, _i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
 _lib.cp_abi_version.argtypes = []
 _lib.cp_abi_version.restype = _i
-ABI_VERSION = 3           # include/cplse.h CPLSE_ABI_VERSION this binding marshals for
+ABI_VERSION = 4           # include/cplse.h CPLSE_ABI_VERSION this binding marshals for
 if _lib.cp_abi_version() != ABI_VERSION:
     raise ImportError("libcplse.so has ABI version %d, this binding needs %d: rebuild it with "
                       "`python lse_pack_stable_b200/build.py`" % (_lib.cp_abi_version(), ABI_VERSION))
@@ -85,10 +86,13 @@ _lib.cp_ipc_import.argtypes = [ctypes.POINTER(IpcHandle), ctypes.POINTER(ctypes.
 _lib.cp_ipc_close.argtypes = [_p]
 _lib.ulysses_seq2head.argtypes = [_p, _p, _i, _i, _i64, _i, _i, _i, _p]
 _lib.ulysses_head2seq.argtypes = [_p, _p, _i, _i, _i64, _i, _i, _i, _p]
+_lib.ulysses_seq2head_pull.argtypes = [_p, _p, _i, _i, _i64, _i, _i, _i, _i, _p]
+_lib.ulysses_head2seq_pull.argtypes = [_p, _p, _i, _i, _i64, _i, _i, _i, _i, _p]
 for _f in ("cp_pack_lse", "cp_lse_materialize", "cp_pack_from_lse", "cp_a2a_local_permute",
            "cp_lse_combine", "cp_pack_permute_combine_fused", "cp_pack_lse_rank",
            "cp_lse_combine_rank", "cp_pull_combine", "cp_ipc_export", "cp_ipc_import",
-           "cp_ipc_close", "ulysses_seq2head", "ulysses_head2seq"):
+           "cp_ipc_close", "ulysses_seq2head", "ulysses_head2seq", "ulysses_seq2head_pull",
+           "ulysses_head2seq_pull"):
     getattr(_lib, _f).restype = _i
 
 
@@ -452,6 +456,61 @@ def ulysses_head2seq(x: torch.Tensor, out: Optional[torch.Tensor] = None,
     _dense(out, "out")
     _check(_lib.ulysses_head2seq(_ptr(x), _ptr(out), W, B, S // W, Hc * W, D, x.element_size(),
                                  _stream(stream)))
+    return out
+
+
+def _ulysses_pull(x: Sequence, out_shape, out: Optional[torch.Tensor], device):
+    """Checks of the W ranks' tensors (same shape, dtype, contiguous) and the
+    output; returns the output and the table of the ranks' addresses."""
+    W = len(x)
+    for r in range(W):
+        _plane(x[r], "x[%d]" % r, 4, x[0])
+        if not _is_dense(x[r]):
+            raise ValueError("x[%d] must be contiguous" % r)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    if out is None:
+        out = torch.empty(out_shape, dtype=x[0].dtype, device=dev)
+    _expect(out, "out", out_shape, x[0].dtype, dev)
+    _dense(out, "out")
+    return out, (ctypes.c_void_p * W)(*[t.data_ptr() for t in x])
+
+
+def _is_dense(t) -> bool:
+    shape, st, want = tuple(t.shape), tuple(t.stride()), 1
+    for n, s in zip(reversed(shape), reversed(st)):
+        if n != 1 and s != want:
+            return False
+        want *= n
+    return True
+
+
+def ulysses_seq2head_pull(x: Sequence, dst: int, out: Optional[torch.Tensor] = None,
+                          device: Optional[torch.device] = None, stream=None) -> torch.Tensor:
+    """Destination `dst` of the seq->head all-to-all across W real ranks: x[r]
+    [B, S/W, H, D] (this device's tensor or a peer's mapped into this process)
+    -> out [B, S, H/W, D]."""
+    W = len(x)
+    if W < 1:
+        raise ValueError("x must list W >= 1 ranks")
+    B, S_l, H, D = x[0].shape
+    out, tab = _ulysses_pull(x, (B, S_l * W, _split(H, W, "H"), D), out, device)
+    _check(_lib.ulysses_seq2head_pull(tab, _ptr(out), W, B, S_l, H, D, out.element_size(), dst,
+                                      _stream(stream)))
+    return out
+
+
+def ulysses_head2seq_pull(x: Sequence, dst: int, out: Optional[torch.Tensor] = None,
+                          device: Optional[torch.device] = None, stream=None) -> torch.Tensor:
+    """Destination `dst` of the head->seq all-to-all across W real ranks: x[r]
+    [B, S, H/W, D] -> out [B, S/W, H, D]."""
+    W = len(x)
+    if W < 1:
+        raise ValueError("x must list W >= 1 ranks")
+    B, S, Hc, D = x[0].shape
+    S_l = _split(S, W, "S")
+    out, tab = _ulysses_pull(x, (B, S_l, Hc * W, D), out, device)
+    _check(_lib.ulysses_head2seq_pull(tab, _ptr(out), W, B, S_l, Hc * W, D, out.element_size(),
+                                      dst, _stream(stream)))
     return out
 
 

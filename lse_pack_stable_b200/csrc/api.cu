@@ -655,6 +655,70 @@ static cp_status ulysses(const void* in, void* out, int W, int B, int64_t S_loca
     return launched(cplse::launch_ulysses(a, static_cast<cudaStream_t>(stream)), what);
 }
 
+static cp_status ulysses_pull(const void* const* in, void* out, int W, int B, int64_t S_local,
+                              int H, int D, int elem_bytes, int dst, void* stream, int mode,
+                              const char* what)
+{
+    if (W < 1) return fail(CP_ERR_ARG, "W must be >= 1 (got %d)", W);
+    if (W > CPLSE_MAX_W) return fail(CP_ERR_UNSUPPORTED, "W = %d exceeds %d", W, CPLSE_MAX_W);
+    if (B < 0 || S_local < 0) return fail(CP_ERR_ARG, "B and S_local must be >= 0");
+    if (B > 65535) return fail(CP_ERR_UNSUPPORTED, "B = %d exceeds 65535", B);
+    if (H < 1 || H % W != 0) return fail(CP_ERR_SHAPE, "H = %d must be a positive multiple of W = %d", H, W);
+    if (D < 1) return fail(CP_ERR_SHAPE, "D must be >= 1");
+    if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8)
+        return fail(CP_ERR_ARG, "elem_bytes must be 1, 2, 4 or 8 (got %d)", elem_bytes);
+    if (dst < 0 || dst >= W) return fail(CP_ERR_ARG, "dst = %d is not a rank of 0..%d", dst, W - 1);
+    const int64_t per_rank = (int64_t)B * H * D * elem_bytes;
+    if (S_local > 0 && per_rank > 0 && S_local > ((int64_t)1 << 62) / ((int64_t)W * per_rank))
+        return fail(CP_ERR_SHAPE, "problem size overflows int64");
+    if (B == 0 || S_local == 0) return ok();
+    TRY(check_null(in, "in"));
+    TRY(check_null(out, "out"));
+    const int64_t bytes = S_local * per_rank;      // one rank's tensor (either layout)
+    const Span outs[1] = {dense_span(out, bytes, "out")};
+    char nm[16];
+    for (int r = 0; r < W; ++r) {
+        snprintf(nm, sizeof nm, "in[%d]", r);
+        TRY(check_null(in[r], nm));
+        const Span ins[1] = {dense_span(in[r], bytes, "in[r]")};
+        TRY(check_no_alias(ins, 1, outs, 1));
+    }
+    {
+        const void* p[1] = {out};
+        const char* n[1] = {"out"};
+        TRY(check_devices(p, n, 1));
+    }
+    for (int r = 0; r < W; ++r) {
+        snprintf(nm, sizeof nm, "in[%d]", r);
+        TRY(check_addressable_ptr(in[r], nm));
+    }
+    cplse::UlyssesArgs a{};
+    a.in = nullptr; a.out = out;
+    a.W = W; a.B = B; a.H = H; a.Hc = H / W;
+    a.S_l = S_local; a.S = S_local * W;
+    a.chunk_bytes = (int64_t)(H / W) * D * elem_bytes;
+    a.nchunks = (int64_t)W * B * S_local;
+    a.mode = mode;
+    a.pull = 1;
+    a.dst = dst;
+    for (int r = 0; r < W; ++r) a.ins[r] = in[r];
+    return launched(cplse::launch_ulysses(a, static_cast<cudaStream_t>(stream)), what);
+}
+
+cp_status ulysses_seq2head_pull(const void* const* in, void* out, int W, int B, int64_t S_local,
+                                int H, int D, int elem_bytes, int dst, void* stream)
+{
+    return ulysses_pull(in, out, W, B, S_local, H, D, elem_bytes, dst, stream, 0,
+                        "ulysses_seq2head_pull");
+}
+
+cp_status ulysses_head2seq_pull(const void* const* in, void* out, int W, int B, int64_t S_local,
+                                int H, int D, int elem_bytes, int dst, void* stream)
+{
+    return ulysses_pull(in, out, W, B, S_local, H, D, elem_bytes, dst, stream, 1,
+                        "ulysses_head2seq_pull");
+}
+
 cp_status ulysses_seq2head(const void* in, void* out, int W, int B, int64_t S_local, int H, int D,
                            int elem_bytes, void* stream)
 {

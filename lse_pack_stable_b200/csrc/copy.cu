@@ -139,7 +139,9 @@ ulysses_kernel(const V* __restrict__ in, V* __restrict__ out, const UlyssesArgs 
 }
 
 // The transforms as 2-D block copies, one grid row per (dst rank j, src rank r)
-// and one grid layer per batch plane b: S_l rows of Hc*D elements each.
+// and one grid layer per batch plane b: S_l rows of Hc*D elements each. In the
+// pull form (one real destination) the grid rows are the source ranks alone,
+// each read through its own base address, and j is the destination.
 //   mode 0: source rows s of in[r][b] at heads j*Hc (row stride H*D) land as
 //           the contiguous rows r*S_l + s of out[j][b];
 //   mode 1: the contiguous source rows j*S_l + s of in[r][b] land as rows s of
@@ -159,20 +161,25 @@ ulysses_block_kernel(const V* __restrict__ in, V* __restrict__ out, const Ulysse
 {
     constexpr int U = kUlyU;
     const int jr = blockIdx.y;
-    const int j = jr / a.W, r = jr - j * a.W;
+    const int j = a.pull ? a.dst : jr / a.W;
+    const int r = a.pull ? jr : jr - j * a.W;
     const int64_t b = blockIdx.z;
     const int64_t rowv = (int64_t)a.W * cv;          // a full H*D row, in vectors
+    const int64_t plane = (int64_t)a.B * a.S_l * rowv;   // one rank's tensor, in vectors
+    // rank r's input and destination j's output
+    const V* in_r = a.pull ? static_cast<const V*>(a.ins[r]) : in + (int64_t)r * plane;
+    V* out_j = a.pull ? out : out + (int64_t)j * plane;
     const V* src;
     V* dst;
     int64_t src_stride, dst_stride;
     if (MODE == 0) {
-        src = in + (((int64_t)r * a.B + b) * a.S_l) * rowv + (int64_t)j * cv;
-        dst = out + (((int64_t)j * a.B + b) * a.S + (int64_t)r * a.S_l) * cv;
+        src = in_r + (b * a.S_l) * rowv + (int64_t)j * cv;
+        dst = out_j + (b * a.S + (int64_t)r * a.S_l) * cv;
         src_stride = rowv;
         dst_stride = cv;
     } else {
-        src = in + (((int64_t)r * a.B + b) * a.S + (int64_t)j * a.S_l) * cv;
-        dst = out + (((int64_t)j * a.B + b) * a.S_l) * rowv + (int64_t)r * cv;
+        src = in_r + (b * a.S + (int64_t)j * a.S_l) * cv;
+        dst = out_j + (b * a.S_l) * rowv + (int64_t)r * cv;
         src_stride = cv;
         dst_stride = rowv;
     }
@@ -201,13 +208,14 @@ cudaError_t launch_ulysses_v(const UlyssesArgs& a, cudaStream_t s)
     if (a.B <= 65535) {
         const int64_t gx = (a.S_l * cv + kCopyThreads * U - 1) / (kCopyThreads * U);
         if (gx <= 0x7fffffff) {
-            dim3 grid((unsigned)gx, (unsigned)(a.W * a.W), (unsigned)a.B);
+            dim3 grid((unsigned)gx, (unsigned)(a.pull ? a.W : a.W * a.W), (unsigned)a.B);
             ulysses_block_kernel<V, MODE><<<grid, kCopyThreads, 0, s>>>(
                 static_cast<const V*>(a.in), static_cast<V*>(a.out), a, cv);
             return cudaGetLastError();
         }
     }
     // more batch planes than a grid layer count allows: one warp per chunk
+    if (a.pull) return cudaErrorInvalidConfiguration;   // the pull form takes B <= 65535
     constexpr int UNR = 4;
     constexpr int K = 2;
     constexpr auto kern = ulysses_kernel<V, MODE, K, UNR>;
@@ -238,7 +246,13 @@ int vector_bytes(int64_t n, const void* p, const void* q)
 template <int MODE>
 cudaError_t launch_ulysses_m(const UlyssesArgs& a, cudaStream_t s)
 {
-    switch (vector_bytes(a.chunk_bytes, a.in, a.out)) {
+    int vb = vector_bytes(a.chunk_bytes, a.in, a.out);
+    if (a.pull)
+        for (int r = 0; r < a.W; ++r) {
+            const int w = vector_bytes(a.chunk_bytes, a.ins[r], a.out);
+            if (w < vb) vb = w;
+        }
+    switch (vb) {
     case 16: return launch_ulysses_v<uint4, MODE>(a, s);
     case 8: return launch_ulysses_v<uint2, MODE>(a, s);
     case 4: return launch_ulysses_v<unsigned int, MODE>(a, s);

@@ -76,6 +76,12 @@ struct UlyssesArgs {
     int64_t chunk_bytes;      // Hc*D*elem_bytes
     int64_t nchunks;
     int mode;                 // 0: seq->head, 1: head->seq
+    // pull form (one real destination rank): rank r's plane at ins[r] (this
+    // GPU's memory or a peer's mapped into this process); out is destination
+    // dst's plane alone
+    int pull;
+    int dst;
+    const void* ins[32];
 };
 
 // the stable merge, fused (from max/sum, in place) or on a received packet:

@@ -24,6 +24,11 @@ fused result, bit for bit:
   it (no owner overwrites them while a peer still reads) orders it against
   the other ranks on the stream, with no host synchronisation and no
   device-side wait in any kernel of this package.
+
+``UlyssesPullExchange`` does the same for the Ulysses layout all-to-alls: each
+rank's sequence shard and head shard are mapped into every rank, and
+destination j's seq->head (head->seq) result is read out of all of them by
+``ulysses_seq2head_pull`` (``ulysses_head2seq_pull``).
 """
 from __future__ import annotations
 
@@ -34,7 +39,7 @@ import torch
 import torch.distributed as dist
 
 from . import (CplseError, IpcHandle, _check, _lib, cp_lse_combine_rank, cp_pack_lse_rank,
-               cp_pull_combine)
+               cp_pull_combine, ulysses_head2seq_pull, ulysses_seq2head_pull)
 
 
 def ipc_export(t: torch.Tensor) -> bytes:
@@ -126,6 +131,50 @@ class A2aExchange:
         return self._combine(self.recv_o, self.recv_lse, out=out, out_lse=out_lse)
 
 
+class PeerMap:
+    """Tensors of this rank shared with every rank of the group: ``table(i)[r]``
+    is rank r's tensor i -- this rank's own tensor, or the peer's mapped into
+    this process (a ``_Plane``). Construction and ``close`` are collective."""
+
+    def __init__(self, tensors, group: Optional[dist.ProcessGroup] = None):
+        self.group = group
+        self.W = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.device = tensors[0].device
+        mine = [ipc_export(t) for t in tensors]
+        every: List = [None] * self.W
+        dist.all_gather_object(every, mine, group=group)
+        self._bases: List[int] = []
+        self._tables: List[List] = [[] for _ in tensors]
+        for r in range(self.W):
+            for i, t in enumerate(tensors):
+                if r == self.rank:
+                    self._tables[i].append(t)
+                else:
+                    base, addr = ipc_import(every[r][i])
+                    self._bases.append(base)
+                    self._tables[i].append(_Plane(addr, t))
+
+    def table(self, i: int) -> List:
+        return self._tables[i]
+
+    def close(self) -> None:
+        """Unmap the peers' tensors, once every rank has finished reading."""
+        if not self._bases:
+            return
+        torch.cuda.synchronize(self.device)
+        dist.barrier(group=self.group)
+        err = None
+        for b in self._bases:
+            try:
+                ipc_close(b)
+            except CplseError as e:  # keep closing the others
+                err = e
+        self._bases = []
+        if err is not None:
+            raise err
+
+
 class PullExchange:
     """This rank's o/max/sum planes, mapped into every rank's process, and the
     pull kernel that merges destination `rank`'s rows from all of them.
@@ -146,25 +195,8 @@ class PullExchange:
         self.smax = torch.empty((T, H), dtype=torch.float32, device=device)
         self.ssum = torch.empty((T, H), dtype=torch.float32, device=device)
         self._flag = torch.zeros(1, dtype=torch.float32, device=device)
-        mine = [ipc_export(t) for t in (self.o, self.smax, self.ssum)]
-        every: List = [None] * self.W
-        dist.all_gather_object(every, mine, group=group)
-        self._bases: List[int] = []
-        self.o_tab, self.m_tab, self.s_tab = [], [], []
-        for r in range(self.W):
-            if r == self.rank:
-                self.o_tab.append(self.o)
-                self.m_tab.append(self.smax)
-                self.s_tab.append(self.ssum)
-                continue
-            planes = []
-            for blob, like in zip(every[r], (self.o, self.smax, self.ssum)):
-                base, addr = ipc_import(blob)
-                self._bases.append(base)
-                planes.append(_Plane(addr, like))
-            self.o_tab.append(planes[0])
-            self.m_tab.append(planes[1])
-            self.s_tab.append(planes[2])
+        self.peers = PeerMap([self.o, self.smax, self.ssum], group)
+        self.o_tab, self.m_tab, self.s_tab = (self.peers.table(i) for i in range(3))
 
     def barrier(self) -> None:
         """Stream-ordered barrier of the group: a one-element all-reduce."""
@@ -180,17 +212,50 @@ class PullExchange:
         return res
 
     def close(self) -> None:
-        """Unmap the peers' planes (collective: every rank first finishes its reads)."""
-        if not self._bases:
-            return
-        torch.cuda.synchronize(self.device)
-        dist.barrier(group=self.group)
-        err = None
-        for b in self._bases:
-            try:
-                ipc_close(b)
-            except CplseError as e:  # keep closing the others
-                err = e
-        self._bases = []
-        if err is not None:
-            raise err
+        self.peers.close()
+
+
+class UlyssesPullExchange:
+    """The Ulysses all-to-alls across real ranks as load/store over NVLink
+    (FastVideo "[perf] Probe H3 chunked all-to-all with direct output slices":
+    all_to_all_4D(x, 2, 1) and its inverse, byte-identical to the NCCL path).
+
+    This rank's sequence shard ``seq`` [B_seq, S/W, H, D] (what seq->head
+    scatters by heads) and head shard ``head`` [B_head, S, H/W, D] (what
+    head->seq gathers back) are allocated here and mapped into every rank;
+    ``seq2head()`` returns this rank's [B_seq, S, H/W, D], ``head2seq()`` its
+    [B_head, S/W, H, D]. Construction is collective."""
+
+    def __init__(self, B_seq: int, B_head: int, S: int, H: int, D: int, dtype: torch.dtype,
+                 device, group: Optional[dist.ProcessGroup] = None):
+        self.group = group
+        self.W = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.device = torch.device(device)
+        S_l = S // self.W
+        if S_l * self.W != S or H % self.W:
+            raise ValueError("S = %d and H = %d must be multiples of W = %d" % (S, H, self.W))
+        self.seq = torch.empty((B_seq, S_l, H, D), dtype=dtype, device=device)
+        self.head = torch.empty((B_head, S, H // self.W, D), dtype=dtype, device=device)
+        self._flag = torch.zeros(1, dtype=torch.float32, device=device)
+        self.peers = PeerMap([self.seq, self.head], group)
+
+    def barrier(self) -> None:
+        dist.all_reduce(self._flag, group=self.group)
+
+    def seq2head(self, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        self.barrier()
+        res = ulysses_seq2head_pull(self.peers.table(0), self.rank, out=out, device=self.device,
+                                    stream=stream)
+        self.barrier()
+        return res
+
+    def head2seq(self, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        self.barrier()
+        res = ulysses_head2seq_pull(self.peers.table(1), self.rank, out=out, device=self.device,
+                                    stream=stream)
+        self.barrier()
+        return res
+
+    def close(self) -> None:
+        self.peers.close()

@@ -41,7 +41,7 @@ def test_only_declared_symbols_are_exported():
 
 
 def test_abi_version():
-    assert cp.abi_version() == cp.ABI_VERSION == 3
+    assert cp.abi_version() == cp.ABI_VERSION == 4
 
 
 # aligned fake addresses: host checks run before any pointer is dereferenced or queried
@@ -263,3 +263,26 @@ def test_ipc_calls_reject_bad_arguments():
     assert "outside" in cp.last_error()
     assert L.cp_ipc_import(None, ctypes.byref(base), ctypes.byref(p)) == cp.CP_ERR_ARG
     assert L.cp_ipc_close(None) == cp.CP_ERR_ARG
+
+
+@pytest.mark.parametrize("kw,status,msg", [
+    (dict(dst=2), cp.CP_ERR_ARG, "dst = 2"),
+    (dict(H=5), cp.CP_ERR_SHAPE, "multiple of W"),
+    (dict(B=70000), cp.CP_ERR_UNSUPPORTED, "65535"),
+    (dict(eb=3), cp.CP_ERR_ARG, "elem_bytes"),
+    (dict(ins=(A, 0)), cp.CP_ERR_ARG, "in[1] is NULL"),
+    (dict(out=A + A // 4 + 16), cp.CP_ERR_ALIAS, "out overlaps input in[r]"),
+])
+def test_ulysses_pull_rejects(kw, status, msg):
+    W, B, S_l, H, D, eb, dst = 2, kw.get("B", 1), 4, kw.get("H", 4), 8, kw.get("eb", 2), kw.get("dst", 0)
+    ins = kw.get("ins", (A, A + A // 4))
+    for f in (L.ulysses_seq2head_pull, L.ulysses_head2seq_pull):
+        assert f(_table(*ins), kw.get("out", 4 * A), W, B, S_l, H, D, eb, dst, None) == status
+        assert msg in cp.last_error()
+
+
+def test_ulysses_pull_reaches_the_device_check():
+    for f in (L.ulysses_seq2head_pull, L.ulysses_head2seq_pull):
+        assert f(_table(A, A + A // 4), 4 * A, 2, 1, 4, 4, 8, 2, 1, None) == cp.CP_ERR_ARG
+        assert _device_check_failed("out")
+        assert f(None, None, 2, 0, 4, 4, 8, 2, 0, None) == cp.CP_OK   # no rows

@@ -235,3 +235,91 @@ def test_pull_exchange_processes_on_one_gpu(world, scatter_dim):
             assert np.array_equal(out_lse.view(np.uint32),
                                   fl[r].cpu().numpy().view(np.uint32)), (r, step)
     assert all(p.exitcode == 0 for p in procs)
+
+
+# --------------------------------------------------------------------- Ulysses across real ranks
+
+@pytest.mark.parametrize("W,B,S_l,H,D,dtype", [(2, 1, 8, 4, 64, torch.bfloat16),
+                                                (4, 3, 16, 8, 128, torch.bfloat16),
+                                                (3, 2, 5, 6, 24, torch.float16),
+                                                (8, 1, 64, 48, 128, torch.bfloat16),
+                                                (4, 2, 7, 4, 3, torch.uint8),
+                                                (2, 2, 9, 2, 5, torch.float32),
+                                                (5, 1, 4, 10, 6, torch.float64)])
+def test_ulysses_pull_equals_the_emulation(W, B, S_l, H, D, dtype, orc):
+    g = torch.Generator().manual_seed(W * 100 + D)
+    x = torch.randint(0, 255, (W, B, S_l, H, D * torch.empty((), dtype=dtype).element_size()),
+                      dtype=torch.uint8, generator=g).view(dtype).cuda()
+    y = cp.ulysses_seq2head(x)
+    ranks = [x[r].clone() for r in range(W)]
+    for j in range(W):
+        yj = cp.ulysses_seq2head_pull(ranks, j)
+        torch.cuda.synchronize()
+        assert torch.equal(yj.view(torch.uint8), y[j].view(torch.uint8)), "seq2head dst %d" % j
+    heads = [y[r].clone() for r in range(W)]
+    for j in range(W):
+        xj = cp.ulysses_head2seq_pull(heads, j)
+        torch.cuda.synchronize()
+        assert torch.equal(xj.view(torch.uint8), x[j].view(torch.uint8)), "head2seq dst %d" % j
+    if dtype == torch.bfloat16:
+        ref = orc.seq2head(x.view(torch.int16).cpu().numpy())
+        assert np.array_equal(y.view(torch.int16).cpu().numpy(), ref)
+
+
+def _uly_worker(rank, world, port, shape, q):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    ex = None
+    try:
+        from lse_pack_stable_b200.exchange import UlyssesPullExchange
+        B, S_l, H, D = shape
+        g = torch.Generator().manual_seed(1234)
+        x = torch.randn((world, B, S_l, H, D), generator=g).to(torch.bfloat16).cuda()
+        ex = UlyssesPullExchange(B, B, S_l * world, H, D, torch.bfloat16, "cuda:0")
+        ex.seq.copy_(x[rank])
+        y = ex.seq2head()
+        ex.head.copy_(y)                      # the head shard that comes back
+        back = ex.head2seq()
+        torch.cuda.synchronize()
+        q.put((rank, y.view(torch.int16).cpu().numpy(), back.view(torch.int16).cpu().numpy()))
+    except Exception as e:  # noqa: BLE001
+        q.put((rank, repr(e), None))
+        raise
+    finally:
+        if ex is not None:
+            ex.close()
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_ulysses_pull_exchange_processes_on_one_gpu(world):
+    import torch.multiprocessing as mp
+    shape = (2, 6, 2 * world, 64)
+    g = torch.Generator().manual_seed(1234)
+    x = torch.randn((world,) + shape, generator=g).to(torch.bfloat16).cuda()
+    y = cp.ulysses_seq2head(x)
+    torch.cuda.synchronize()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_uly_worker, args=(r, world, port, shape, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(world):
+        r, yr, back = q.get(timeout=240)
+        got[r] = (yr, back)
+    for p in procs:
+        p.join(120)
+    for r in range(world):
+        yr, back = got[r]
+        assert not isinstance(yr, str), yr
+        assert np.array_equal(yr, y[r].view(torch.int16).cpu().numpy()), "seq2head rank %d" % r
+        assert np.array_equal(back, x[r].view(torch.int16).cpu().numpy()), "round trip rank %d" % r
+    assert all(p.exitcode == 0 for p in procs)
