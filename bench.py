@@ -734,11 +734,79 @@ def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
                      "hbm_peak_GB/s": peak, "hbm_peak_source": peak_source(peak_kind)},
         "cpu_baseline": None, "breakdown": None, "per_config": None,
     }
+    if wl.name == "ulysses":
+        line["ulysses_exchange"] = measure_ulysses_exchange(wl, dev, stream, K, Wm, barrier, world)
     if rank == 0:
         print(json.dumps(line), flush=True)
     torch.cuda.synchronize()
     pull.close()
     return 0
+
+
+def all_to_all_4d_nccl(x, scatter_dim, gather_dim, world, out_shape):
+    """The NCCL all-to-all of the Ulysses layout that the load/store exchange
+    must match byte for byte: torch reshapes around all_to_all_single
+    (seq->head: scatter_dim 2, gather_dim 1; head->seq: the inverse)."""
+    import torch
+    import torch.distributed as dist
+    B, A1, A2, D = x.shape
+    if scatter_dim == 2:            # [B, S/W, H, D] -> send [W, B, S/W, H/W, D]
+        send = x.reshape(B, A1, world, A2 // world, D).permute(2, 0, 1, 3, 4).contiguous()
+    else:                           # [B, S, H/W, D] -> send [W, B, S/W, H/W, D]
+        send = x.reshape(B, world, A1 // world, A2, D).permute(1, 0, 2, 3, 4).contiguous()
+    recv = torch.empty_like(send)
+    dist.all_to_all_single(recv.view(torch.uint8), send.view(torch.uint8))
+    if gather_dim == 1:             # [W, B, S/W, Hc, D] -> [B, S, Hc, D]
+        return recv.permute(1, 0, 2, 3, 4).reshape(out_shape)
+    return recv.permute(1, 2, 0, 3, 4).reshape(out_shape)   # -> [B, S/W, H, D]
+
+
+def measure_ulysses_exchange(wl, dev, stream, K, Wm, barrier, world):
+    """The Ulysses transforms across the N GPUs: q/k/v (B = 3) seq->head and o
+    (B = 1) head->seq by load/store over NVLink (UlyssesPullExchange), against
+    the NCCL all_to_all_4D; both must agree bit for bit."""
+    import torch
+    import torch.distributed as dist
+    from lse_pack_stable_b200.exchange import UlyssesPullExchange
+
+    rank = dist.get_rank()
+    S, H, D = wl.T, wl.H, wl.D
+    Bq, Bo = wl.ulysses_B
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float16
+    ex = UlyssesPullExchange(Bq, Bo, S, H, D, tdt, dev)
+    wlr = synth.Workload(**{**wl.__dict__, "W": world})
+    ex.seq.view(torch.int16).copy_(torch.from_numpy(
+        synth.ulysses_seq_block(wlr, rank).view(np.int16)))
+    ex.head.view(torch.int16).copy_(torch.from_numpy(
+        synth.ulysses_head_block(wlr, rank).view(np.int16)))
+    y = torch.empty((Bq, S, H // world, D), dtype=tdt, device=dev)
+    z = torch.empty((Bo, S // world, H, D), dtype=tdt, device=dev)
+    ex.seq2head(out=y)
+    ex.head2seq(out=z)
+    y_ref = all_to_all_4d_nccl(ex.seq, 2, 1, world, y.shape)
+    z_ref = all_to_all_4d_nccl(ex.head, 1, 2, world, z.shape)
+    torch.cuda.synchronize()
+    same = torch.tensor([float(torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+                               and torch.equal(z.view(torch.int16), z_ref.view(torch.int16)))],
+                        device=dev)
+    dist.all_reduce(same, op=dist.ReduceOp.MIN)
+    t = {}
+    t["seq2head_pull"] = time_back_to_back(lambda i: ex.seq2head(out=y), stream, K, Wm, barrier)
+    t["head2seq_pull"] = time_back_to_back(lambda i: ex.head2seq(out=z), stream, K, Wm, barrier)
+    t["seq2head_nccl"] = time_back_to_back(
+        lambda i: all_to_all_4d_nccl(ex.seq, 2, 1, world, y.shape), stream, K, Wm, barrier)
+    t["head2seq_nccl"] = time_back_to_back(
+        lambda i: all_to_all_4d_nccl(ex.head, 1, 2, world, z.shape), stream, K, Wm, barrier)
+    names = list(t)
+    ms = dict(zip(names, reduce_max([t[n] for n in names], world, dev)))
+    torch.cuda.synchronize()
+    ex.close()
+    return {"pull_equals_nccl": bool(same.item() == 1.0),
+            **{n + "_us": round(ms[n] / K * 1e3, 3) for n in names},
+            "bytes_per_rank": {"seq2head": ex.seq.numel() * ex.seq.element_size(),
+                               "head2seq": ex.head.numel() * ex.head.element_size()},
+            "note": "q/k/v [3, S/W, H, D] seq->head and o [1, S, H/W, D] head->seq per rank; "
+                    "NCCL: all_to_all_single between torch reshapes"}
 
 
 def measure_e2e(cp, wl, inp, stream, dev, K, Wm, barrier, world):

@@ -115,3 +115,54 @@ def test_a2a_exchange_over_gloo(world, scatter_dim):
         ob, ol = got[j]
         assert np.array_equal(ob.view(np.uint16), ref[j]), "payload of destination %d" % j
         assert np.array_equal(ol.view(np.uint32), ref_lse[j].astype(np.float32).view(np.uint32))
+
+
+def _uly_worker(rank, world, port, q):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        g = torch.Generator().manual_seed(99)
+        B, S_l, H, D = 2, 5, 2 * world, 8
+        x = torch.randint(-30000, 30000, (world, B, S_l, H, D), dtype=torch.int16, generator=g)
+        y = bench.all_to_all_4d_nccl(x[rank].view(torch.bfloat16), 2, 1, world,
+                                     (B, S_l * world, H // world, D))
+        h = torch.randint(-30000, 30000, (world, B, S_l * world, H // world, D), dtype=torch.int16,
+                          generator=g)
+        z = bench.all_to_all_4d_nccl(h[rank].view(torch.bfloat16), 1, 2, world, (B, S_l, H, D))
+        q.put((rank, y.view(torch.int16).numpy().copy(), z.view(torch.int16).numpy().copy(),
+               x.numpy(), h.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_nccl_style_all_to_all_4d_reference(world):
+    """The bench's NCCL-path reference for the Ulysses exchange (torch reshapes
+    around all_to_all_single), run over gloo, equals the oracle's transforms."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    orc = oracle.get()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_uly_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(world):
+        r, y, z, x, h = q.get(timeout=120)
+        got[r] = (y, z)
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    ref_y = orc.seq2head(x)
+    ref_z = orc.head2seq(h)
+    for r in range(world):
+        assert np.array_equal(got[r][0], ref_y[r]), "seq->head rank %d" % r
+        assert np.array_equal(got[r][1], ref_z[r]), "head->seq rank %d" % r
