@@ -480,7 +480,7 @@ def time_back_to_back(step, stream, K, Wm, barrier):
     return a.elapsed_time(b)
 
 
-def time_launches(fn, stream, reps, warm=3):
+def time_launches(fn, stream, reps, warm=3, hold_ms=None):
     """Device time (ms) of each of `reps` calls, each bracketed by its own event
     pair on the launching stream; calls follow each other with no host wait,
     one synchronisation at the end."""
@@ -490,7 +490,7 @@ def time_launches(fn, stream, reps, warm=3):
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(reps)]
-    hold_device(stream, max(2.0, 0.2 * reps))
+    hold_device(stream, hold_ms if hold_ms is not None else max(2.0, 0.2 * reps))
     for i in range(reps):
         ev[i][0].record(stream)
         fn(i)
@@ -962,8 +962,8 @@ def measure_breakdown(cp, wl, sets, stream, dev, peak):
     rv = [(torch.empty_like(pk[0][0]), torch.empty_like(pk[0][1])) for _ in range(nb)]
     res = {}
 
-    def rec(name, fn, nbytes, reps=20):
-        res[name] = launch_stats(time_launches(fn, stream, reps), nbytes, peak)
+    def rec(name, fn, nbytes, reps=20, hold_ms=None):
+        res[name] = launch_stats(time_launches(fn, stream, reps, hold_ms=hold_ms), nbytes, peak)
 
     def pack(i):
         cp.cp_pack_lse(*sets[i % n][:3], pkt_o=pk[i % nb][0], pkt_lse=pk[i % nb][1], stream=stream)
@@ -1003,6 +1003,25 @@ def measure_breakdown(cp, wl, sets, stream, dev, peak):
                                                        stream=stream),
             wl.fused_bytes())
         del touts
+    # the pull kernel of the exchange across GPUs, here reading the W planes of
+    # this GPU's own input (HBM, not NVLink): every destination, one launch each
+    import ctypes
+    sh = stream.cuda_stream
+    pull_args = []
+    for st in sets:
+        oi, mi, si, out, ol = st
+        tabs = [(ctypes.c_void_p * W)(*[t[r].data_ptr() for r in range(W)]) for t in (oi, mi, si)]
+        pull_args.append([(tabs[0], cp._strides_plane(oi[0]), tabs[1], cp._strides_plane(mi[0]),
+                           tabs[2], cp._strides_plane(si[0]), W, T, H, D, cp._dtype(oi), 1, j,
+                           out[j].data_ptr(), ol[j].data_ptr(), sh) for j in range(W)])
+
+    def pull_all(i):
+        for args in pull_args[i % n]:
+            st_ = cp._lib.cp_pull_combine(*args)
+            if st_ != 0:
+                raise cp.CplseError(st_, cp.last_error())
+    rec("pull_all_destinations", pull_all, wl.fused_bytes(), hold_ms=max(2.0, 0.1 * 20 * W))
+    del pull_args
     # context for the fused share at this size: a plain device-to-device copy
     # moving the fused kernel's byte count (half read, half written), timed the
     # same way, its source rotating over the same sets
