@@ -6,8 +6,11 @@ checks sampled output rows one by one: for each sampled (t, h) the generator
 regenerates that row's W partial outputs and statistics, and the oracle merges
 them (``fused_gathered``). Properties that hold at any size are checked over
 every element on the device: the unfused pack -> all-to-all -> combine chain
-equals the fused kernel bit for bit. The Ulysses transforms are compared with
-the oracle in full.
+equals the fused kernel bit for bit, and so do the entry points of the
+exchange across GPUs (the pull kernel for every destination, one rank's pack,
+one destination's combine), run here on the W planes of one GPU. The Ulysses
+transforms are compared with the oracle in full, and their pull form with
+them.
 """
 from __future__ import annotations
 
@@ -84,9 +87,25 @@ def test_fullsize_fused_and_chain(name, orc):
     check_combined(got, got_lse, ref, ref_lse, ref_r, wl.dtype, W,
                    extra_lse_tol=lse_member_tol(rm, rs))
 
+    # the pull kernel of the exchange across GPUs, every destination, reading the
+    # W planes of this GPU's input: destination j of the fused result, bit for bit
+    planes = ([o[r] for r in range(W)], [m[r] for r in range(W)], [s[r] for r in range(W)])
+    for jj in range(W):
+        po, pl_ = cp.cp_pull_combine(*planes, jj)
+        torch.cuda.synchronize()
+        assert torch.equal(po.view(torch.int16), out[jj].view(torch.int16)), "pull, dst %d" % jj
+        assert torch.equal(pl_.view(torch.int32), out_lse[jj].view(torch.int32))
+        del po, pl_
+
     # unfused chain on the full problem, then back to the sampled rows
     pkt, pl = cp.cp_pack_lse(o, m, s, scatter_dim=1)
     torch.cuda.synchronize()
+    for r in (0, W - 1):          # one real rank's pack: plane r of the packet
+        po, plr = cp.cp_pack_lse_rank(o[r], m[r], s[r], W)
+        torch.cuda.synchronize()
+        assert torch.equal(po.view(torch.int16), pkt[r].view(torch.int16)), "rank pack %d" % r
+        assert torch.equal(plr.view(torch.int32), pl[r].view(torch.int32))
+        del po, plr
     ri = torch.arange(W, device="cuda")[:, None]
     pk_rows = pkt[ri, ji[None], ti[None], hci[None]]          # [W, n, D]
     assert np.array_equal(host_bits(pk_rows), ro), "packet payload differs from the inputs"
@@ -103,6 +122,12 @@ def test_fullsize_fused_and_chain(name, orc):
     torch.cuda.synchronize()
     assert torch.equal(co.view(torch.int16), out.view(torch.int16)), "chain != fused"
     assert torch.equal(cl.view(torch.int32), out_lse.view(torch.int32)), "chain LSE != fused"
+    for jj in (0, W - 1):         # one real destination's combine
+        oj, lj = cp.cp_lse_combine_rank(recv[jj], recv_l[jj])
+        torch.cuda.synchronize()
+        assert torch.equal(oj.view(torch.int16), out[jj].view(torch.int16)), "rank combine %d" % jj
+        assert torch.equal(lj.view(torch.int32), out_lse[jj].view(torch.int32))
+        del oj, lj
     del recv, recv_l, co, cl, out, out_lse, m, s
     torch.cuda.empty_cache()
 
@@ -146,6 +171,14 @@ def test_fullsize_ulysses(orc):
     back = cp.ulysses_head2seq(y)
     torch.cuda.synchronize()
     assert torch.equal(back.view(torch.int16), xd.view(torch.int16))
+    # the load/store exchange across GPUs, every destination, from this GPU's planes
+    for j in range(W):
+        yj = cp.ulysses_seq2head_pull([xd[r] for r in range(W)], j)
+        bj = cp.ulysses_head2seq_pull([y[r] for r in range(W)], j)
+        torch.cuda.synchronize()
+        assert torch.equal(yj.view(torch.int16), y[j].view(torch.int16)), "seq2head pull %d" % j
+        assert torch.equal(bj.view(torch.int16), xd[j].view(torch.int16)), "head2seq pull %d" % j
+        del yj, bj
     del xd, y, back
     xh = np.stack([synth.ulysses_head_block(wl, r) for r in range(W)])      # [W,1,S,Hc,D]
     hd = torch.from_numpy(xh.view(np.int16)).cuda().view(torch.bfloat16)
