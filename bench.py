@@ -1004,24 +1004,33 @@ def measure_breakdown(cp, wl, sets, stream, dev, peak):
             wl.fused_bytes())
         del touts
     # the pull kernel of the exchange across GPUs, here reading the W planes of
-    # this GPU's own input (HBM, not NVLink): every destination, one launch each
+    # this GPU's own input (HBM, not NVLink): every destination at once, one
+    # launch each on its own stream, as the W GPUs of a real exchange read every
+    # rank's memory concurrently
     import ctypes
-    sh = stream.cuda_stream
+    pstreams = [torch.cuda.Stream(dev) for _ in range(W)]
+    forked, joined = torch.cuda.Event(), [torch.cuda.Event() for _ in range(W)]
     pull_args = []
     for st in sets:
         oi, mi, si, out, ol = st
         tabs = [(ctypes.c_void_p * W)(*[t[r].data_ptr() for r in range(W)]) for t in (oi, mi, si)]
         pull_args.append([(tabs[0], cp._strides_plane(oi[0]), tabs[1], cp._strides_plane(mi[0]),
                            tabs[2], cp._strides_plane(si[0]), W, T, H, D, cp._dtype(oi), 1, j,
-                           out[j].data_ptr(), ol[j].data_ptr(), sh) for j in range(W)])
+                           out[j].data_ptr(), ol[j].data_ptr(), pstreams[j].cuda_stream)
+                          for j in range(W)])
 
     def pull_all(i):
-        for args in pull_args[i % n]:
+        forked.record(stream)
+        for j, args in enumerate(pull_args[i % n]):
+            pstreams[j].wait_event(forked)
             st_ = cp._lib.cp_pull_combine(*args)
             if st_ != 0:
                 raise cp.CplseError(st_, cp.last_error())
+            joined[j].record(pstreams[j])
+        for ev in joined:
+            stream.wait_event(ev)
     rec("pull_all_destinations", pull_all, wl.fused_bytes(), hold_ms=max(2.0, 0.1 * 20 * W))
-    del pull_args
+    del pull_args, pstreams
     # context for the fused share at this size: a plain device-to-device copy
     # moving the fused kernel's byte count (half read, half written), timed the
     # same way, its source rotating over the same sets

@@ -185,11 +185,7 @@ cudaError_t launch_pull_inst(const PullArgs& a, cudaStream_t s)
         const cudaError_t e = resident_blocks<kern>(kPullThreads, 0, per_sm);
         if (e != cudaSuccess) return e;
     }
-    const int64_t nchunks = (a.rows + 31) / 32;
-    int64_t blocks = (nchunks + kPullThreads / 32 - 1) / (kPullThreads / 32);
-    const int64_t cap = (int64_t)per_sm * sm_count();
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
+    const int64_t blocks = merge_grid(a.rows, kPullThreads, per_sm, U * (32 / G));
     return launch_pdl(kern, (unsigned)blocks, kPullThreads, 0, s, a);
 }
 

@@ -288,6 +288,22 @@ rowcombine_kernel(const CombineArgs a)
     }
 }
 
+// Blocks of a merge grid: enough warps that each gets at least `min_rows`
+// output rows (one batch of loads in flight; ChunkPlan then splits the rows
+// evenly), at most what is resident on the whole GPU at once. A problem with
+// few rows thus still spreads over every SM instead of giving each of a few
+// warps a whole 32-row chunk.
+inline int64_t merge_grid(int64_t rows, int threads, int per_sm, int min_rows)
+{
+    const int64_t wpb = threads / 32;
+    const int64_t warps = (rows + min_rows - 1) / min_rows;
+    int64_t blocks = (warps + wpb - 1) / wpb;
+    const int64_t cap = (int64_t)per_sm * sm_count();
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    return blocks;
+}
+
 // Launch with programmatic stream serialization: back-to-back launches overlap
 // the next grid's scheduling with this one's drain. Every merge kernel opens
 // with griddepcontrol.wait, so none reads memory before the previous kernel in
@@ -338,12 +354,8 @@ cudaError_t launch_rowcombine_inst(const CombineArgs& a, cudaStream_t s)
         const cudaError_t e = resident_blocks<kern>(kCombineThreads, 0, per_sm);
         if (e != cudaSuccess) return e;
     }
-    const int64_t nchunks = (a.rows + 31) / 32;
-    const int64_t warps_per_block = kCombineThreads / 32;
-    int64_t blocks = (nchunks + warps_per_block - 1) / warps_per_block;
-    const int64_t cap = (int64_t)per_sm * sm_count();
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
+    // one batch of loads: U steps of 32/G rows
+    const int64_t blocks = merge_grid(a.rows, kCombineThreads, per_sm, U * (32 / G));
     return launch_pdl(kern, (unsigned)blocks, kCombineThreads, 0, s, a);
 }
 

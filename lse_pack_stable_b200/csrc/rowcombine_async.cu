@@ -31,11 +31,8 @@ cudaError_t launch_async_inst(const CombineArgs& a, cudaStream_t s)
         const cudaError_t e = resident_blocks<kern>(kAsyncThreads, smem, per_sm);
         if (e != cudaSuccess) return e;
     }
-    const int64_t nchunks = (a.rows + 31) / 32;
-    int64_t blocks = (nchunks + kAsyncThreads / 32 - 1) / (kAsyncThreads / 32);
-    const int64_t cap = (int64_t)per_sm * sm_count();
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
+    // the ring's groups in flight: NST-1 steps of 32/G rows
+    const int64_t blocks = merge_grid(a.rows, kAsyncThreads, per_sm, (NST - 1) * (32 / G));
     return launch_pdl(kern, (unsigned)blocks, kAsyncThreads, smem, s, a);
 }
 
