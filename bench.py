@@ -1046,7 +1046,29 @@ def measure_breakdown(cp, wl, sets, stream, dev, peak):
         rec("ulysses_seq2head", lambda i: cp.ulysses_seq2head(xs[i % 2], out=ys[i % 2],
                                                               stream=stream),
             2 * xs[0].numel() * 2)
-        del xs, ys
+        # the load/store exchange across GPUs: every destination at once, one
+        # launch each on its own stream, from the W planes of this GPU
+        ustreams = [torch.cuda.Stream(dev) for _ in range(W)]
+        ufork, ujoin = torch.cuda.Event(), [torch.cuda.Event() for _ in range(W)]
+        uargs = []
+        for x, y in zip(xs, ys):
+            tab = (ctypes.c_void_p * W)(*[x[r].data_ptr() for r in range(W)])
+            uargs.append([(tab, y[j].data_ptr(), W, 3, S_l, H, D, 2, j, ustreams[j].cuda_stream)
+                          for j in range(W)])
+
+        def uly_pull_all(i):
+            ufork.record(stream)
+            for j, args in enumerate(uargs[i % 2]):
+                ustreams[j].wait_event(ufork)
+                st_ = cp._lib.ulysses_seq2head_pull(*args)
+                if st_ != 0:
+                    raise cp.CplseError(st_, cp.last_error())
+                ujoin[j].record(ustreams[j])
+            for ev in ujoin:
+                stream.wait_event(ev)
+        rec("ulysses_seq2head_pull_all_destinations", uly_pull_all, 2 * xs[0].numel() * 2,
+            hold_ms=max(2.0, 0.1 * 20 * W))
+        del xs, ys, uargs, ustreams
         hs = [torch.empty((W, 1, T, Hc, D), dtype=tdt, device=dev).normal_() for _ in range(2)]
         gs = [torch.empty((W, 1, S_l, H, D), dtype=tdt, device=dev) for _ in range(2)]
         rec("ulysses_head2seq", lambda i: cp.ulysses_head2seq(hs[i % 2], out=gs[i % 2],
