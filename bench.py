@@ -520,7 +520,7 @@ def measure_workload(cp, wl, dev, stream, args, world, barrier, peak, peak_kind,
     bytes_per_call = wl.fused_bytes()
     K, Wm = max(1, args.steps), max(3, args.warmup)
 
-    clocks = ClockSampler(local_rank)
+    clocks = ClockSampler(dev.index)
     clocks.start()
     total_ms = time_back_to_back(step, stream, K, Wm, barrier)
     launch_ms = time_launches(step, stream, max(ROOFLINE_LAUNCHES, args.launches))
@@ -569,15 +569,19 @@ def run_ours(args):
     import lse_pack_stable_b200 as cp
 
     rank, local_rank, world = env_rank()
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
+    # one process per GPU; with fewer GPUs than ranks (the host-collective test
+    # of this path) ranks share devices
+    device_index = local_rank % torch.cuda.device_count()
+    torch.cuda.set_device(device_index)
+    dev = torch.device("cuda", device_index)
     peak, peak_kind = measured_peak()
     if world > 1:
         # the communicator's own log stays on; no NVLink multicast (NVLS) objects
         os.environ.setdefault("NCCL_DEBUG", "INFO")
         os.environ.setdefault("NCCL_NVLS_ENABLE", "0")
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        backend = os.environ.get("CPLSE_BENCH_BACKEND", "nccl")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120),
+                                device_id=dev if backend == "nccl" else None)
         try:
             return run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind)
         finally:
@@ -642,6 +646,8 @@ def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
     from lse_pack_stable_b200.exchange import A2aExchange, PullExchange
 
     wl = workload_for(args.config, world)
+    if args.tokens > 0:
+        wl = synth.Workload(**{**wl.__dict__, "T": args.tokens})
     T, H, D, Hc = wl.T, wl.H, wl.D, wl.H // world
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float16
     stream = torch.cuda.current_stream(dev)
@@ -680,7 +686,7 @@ def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
                         device=dev)
     dist.all_reduce(same, op=dist.ReduceOp.MIN)
 
-    clocks = ClockSampler(local_rank)
+    clocks = ClockSampler(dev.index)
     clocks.start()
     pull_ms = time_back_to_back(lambda i: pull(out_p, lse_p), stream, K, Wm, barrier)
     a2a_ms = time_back_to_back(lambda i: a2a(pull.o, pull.smax, pull.ssum, out_a, lse_a), stream,
