@@ -131,6 +131,18 @@ class A2aExchange:
         return self._combine(self.recv_o, self.recv_lse, out=out, out_lse=out_lse)
 
 
+def _stream_barrier(flag: torch.Tensor, group, stream=None) -> None:
+    """Every rank of `group` reaches this point on `stream` before anything
+    enqueued on `stream` afterwards runs: a one-element all-reduce issued with
+    `stream` current (torch orders a collective after the current stream's
+    work and makes that stream wait for it)."""
+    if stream is None:
+        dist.all_reduce(flag, group=group)
+        return
+    with torch.cuda.stream(stream):
+        dist.all_reduce(flag, group=group)
+
+
 class PeerMap:
     """Tensors of this rank shared with every rank of the group: ``table(i)[r]``
     is rank r's tensor i -- this rank's own tensor, or the peer's mapped into
@@ -181,7 +193,9 @@ class PullExchange:
 
     The producer writes this rank's partial output into ``o``, ``smax`` and
     ``ssum`` (allocated here); each call then returns this destination's
-    combined rows. Construction is collective (every rank of the group)."""
+    combined rows. Construction is collective (every rank of the group), and
+    so is ``close()``, which every rank calls before dropping the object: the
+    planes stay allocated until then, as peers may still read them."""
 
     def __init__(self, T: int, H: int, D: int, dtype: torch.dtype, device,
                  group: Optional[dist.ProcessGroup] = None, scatter_dim: int = 1):
@@ -198,17 +212,18 @@ class PullExchange:
         self.peers = PeerMap([self.o, self.smax, self.ssum], group)
         self.o_tab, self.m_tab, self.s_tab = (self.peers.table(i) for i in range(3))
 
-    def barrier(self) -> None:
-        """Stream-ordered barrier of the group: a one-element all-reduce."""
-        dist.all_reduce(self._flag, group=self.group)
+    def barrier(self, stream=None) -> None:
+        """Barrier of the group, ordered on `stream` (default: the current
+        stream): a one-element all-reduce issued from that stream."""
+        _stream_barrier(self._flag, self.group, stream)
 
     def __call__(self, out: Optional[torch.Tensor] = None,
                  out_lse: Optional[torch.Tensor] = None, stream=None):
-        self.barrier()          # every rank has written its planes
+        self.barrier(stream)    # every rank has written its planes
         res = cp_pull_combine(self.o_tab, self.m_tab, self.s_tab, self.rank,
                               scatter_dim=self.scatter_dim, out=out, out_lse=out_lse,
                               device=self.device, stream=stream)
-        self.barrier()          # no rank overwrites its planes while a peer reads them
+        self.barrier(stream)    # no rank overwrites its planes while a peer reads them
         return res
 
     def close(self) -> None:
@@ -240,21 +255,21 @@ class UlyssesPullExchange:
         self._flag = torch.zeros(1, dtype=torch.float32, device=device)
         self.peers = PeerMap([self.seq, self.head], group)
 
-    def barrier(self) -> None:
-        dist.all_reduce(self._flag, group=self.group)
+    def barrier(self, stream=None) -> None:
+        _stream_barrier(self._flag, self.group, stream)
 
     def seq2head(self, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-        self.barrier()
+        self.barrier(stream)
         res = ulysses_seq2head_pull(self.peers.table(0), self.rank, out=out, device=self.device,
                                     stream=stream)
-        self.barrier()
+        self.barrier(stream)
         return res
 
     def head2seq(self, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-        self.barrier()
+        self.barrier(stream)
         res = ulysses_head2seq_pull(self.peers.table(1), self.rank, out=out, device=self.device,
                                     stream=stream)
-        self.barrier()
+        self.barrier(stream)
         return res
 
     def close(self) -> None:
