@@ -187,12 +187,17 @@ def _pull_worker(rank, world, port, wl, scatter_dim, q):
         ex = PullExchange(wl.T, wl.H, wl.D, pay(o[:1], wl.dtype).dtype, "cuda:0",
                           scatter_dim=scatter_dim)
         res = []
+        side = torch.cuda.Stream()
         for step in range(2):             # the second step overwrites the planes
             scale = 1 if step == 0 else -1
             ex.o.copy_(pay(o[rank], wl.dtype) * scale)
             ex.smax.copy_(f32(m[rank]))
             ex.ssum.copy_(f32(s[rank]))
-            out, out_lse = ex()
+            if step == 0:
+                out, out_lse = ex()
+            else:                         # on a side stream: the barriers order that stream
+                side.wait_stream(torch.cuda.current_stream())
+                out, out_lse = ex(stream=side)
             torch.cuda.synchronize()
             res.append((out.view(torch.int16).cpu().numpy(), out_lse.cpu().numpy()))
         q.put((rank, res))
