@@ -16,9 +16,10 @@
 // Work split: the register-staged scheme of rowcombine.cuh. A warp owns chunks
 // of 32 output rows. Phase A: lane i forms the W LSE values of row i (one
 // coalesced float from each rank's max and sum plane) and the merge weights
-// (merge_weights, the arithmetic every merge kernel shares). Phase B: G lanes
-// cover a row with 16-byte vectors; every rank's vector of U steps is loaded
-// before any is used, accumulated in fp32 in rank order, rounded and stored.
+// (merge_weights, the arithmetic every merge kernel shares), which it writes
+// to a per-warp table in shared memory. Phase B: G lanes cover a row with
+// 16-byte vectors; every rank's vector of U steps is loaded before any is
+// used, accumulated in fp32 in rank order, rounded and stored.
 // A weight-0 contribution is neither loaded nor added (-0.0 stands in).
 //
 // No bulk copies, no TMA and no multicast: every remote byte arrives through
@@ -36,14 +37,20 @@ namespace {
 constexpr int kPullThreads = 128;
 
 template <typename P, int WMAX, int G, int VPL, int U>
-__global__ void __launch_bounds__(kPullThreads) pull_combine_kernel(const PullArgs a)
+__global__ void __launch_bounds__(kPullThreads, merge_min_blocks<VPL>())
+pull_combine_kernel(const PullArgs a)
 {
     constexpr int RPI = 32 / G;          // rows per step
     constexpr int STEPS = 32 / RPI;      // steps per chunk
-    constexpr int RB = WMAX < 16 ? WMAX : 16;   // ranks loaded at once
+    // ranks loaded at once: 16 vectors in flight per lane per batch
+    constexpr int RB = WMAX < 16 / VPL ? WMAX : 16 / VPL;
+    constexpr int WS = (WMAX + 3) / 4 * 4;
     static_assert(STEPS % U == 0, "U must divide the steps of a chunk");
+    // per-warp row table: the weights of the chunk's 32 rows
+    __shared__ __align__(16) float wtab[kPullThreads / 32][32][WS];
 
     const int lane = threadIdx.x & 31;
+    const int wib = threadIdx.x >> 5;
     const int sub = lane / G;
     const int gl = lane % G;
     const int64_t warp = ((int64_t)blockIdx.x * kPullThreads + threadIdx.x) >> 5;
@@ -76,37 +83,50 @@ __global__ void __launch_bounds__(kPullThreads) pull_combine_kernel(const PullAr
         const int64_t src_row = t * a.so_t + h * a.so_h;
         const int64_t mo = t * a.sm_t + h * a.sm_h;
         const int64_t so = t * a.ss_t + h * a.ss_h;
-        float lse[WMAX];
+        uint32_t vmask = 0;               // bit r: contribution r has a nonzero weight
+        bool row_dead;
+        {
+            float lse[WMAX];
 #pragma unroll
-        for (int r = 0; r < WMAX; ++r) {
-            float m = -INFINITY, sm = 0.f;
-            if (qv && r < a.W) {
-                m = ld_stream(a.smax[r] + mo);
-                sm = ld_stream(a.ssum[r] + so);
+            for (int r = 0; r < WMAX; ++r) {
+                float m = -INFINITY, sm = 0.f;
+                if (qv && r < a.W) {
+                    m = ld_stream(a.smax[r] + mo);
+                    sm = ld_stream(a.ssum[r] + so);
+                }
+                // invalid statistic: non-finite max, non-finite sum, or sum <= 0
+                const bool ok = isfinite(m) && isfinite(sm) && sm > 0.f;
+                lse[r] = ok ? m + logf(sm) : -INFINITY;
             }
-            // invalid statistic: non-finite max, non-finite sum, or sum <= 0
-            const bool ok = isfinite(m) && isfinite(sm) && sm > 0.f;
-            lse[r] = ok ? m + logf(sm) : -INFINITY;
+            float w[WS];
+            float L;
+            row_dead = !merge_weights(lse, w, L);
+            if (qv) st_stream(a.out_lse + q, L);
+#pragma unroll
+            for (int r = 0; r < WMAX; ++r) vmask |= (w[r] != 0.f ? 1u : 0u) << r;
+            __syncwarp();                 // the previous chunk's table is read
+#pragma unroll
+            for (int r = 0; r < WS; r += 4)
+                *reinterpret_cast<float4*>(&wtab[wib][lane][r]) =
+                    make_float4(w[r], w[r + 1], w[r + 2], w[r + 3]);
+            __syncwarp();                 // the table is visible to the warp
         }
-        float w[WMAX];
-        float L;
-        const bool row_dead = !merge_weights(lse, w, L);
-        if (qv) st_stream(a.out_lse + q, L);
 
-        // ---------------- phase B: G lanes per row
+        // ---------------- phase B: G lanes per row (weights from the table)
 #pragma unroll 1
         for (int s0 = 0; s0 < STEPS; s0 += U) {
             int64_t sb[U];
             bool rv[U], dead[U];
-            float ws[U][WMAX];
+            uint32_t msk[U];
+            int kk[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int k = (s0 + u) * RPI + sub;
+                kk[u] = k;
                 sb[u] = __shfl_sync(kFull, src_row, k);
                 dead[u] = __shfl_sync(kFull, (int)row_dead, k) != 0;
+                msk[u] = __shfl_sync(kFull, vmask, k);
                 rv[u] = k < cn;
-#pragma unroll
-                for (int r = 0; r < WMAX; ++r) ws[u][r] = __shfl_sync(kFull, w[r], k);
             }
             float acc[U][VPL][8];
 #pragma unroll
@@ -116,8 +136,8 @@ __global__ void __launch_bounds__(kPullThreads) pull_combine_kernel(const PullAr
 #pragma unroll
                     for (int x = 0; x < 8; ++x) acc[u][e][x] = -0.f;
 
-#pragma unroll
-            for (int r0 = 0; r0 < WMAX; r0 += RB) {
+#pragma unroll 1
+            for (int r0 = 0; r0 < WMAX; r0 += RB) {   // one batch of ranks at a time
                 uint4 v[U][VPL][RB];
 #pragma unroll
                 for (int u = 0; u < U; ++u)
@@ -127,7 +147,7 @@ __global__ void __launch_bounds__(kPullThreads) pull_combine_kernel(const PullAr
 #pragma unroll
                         for (int rr = 0; rr < RB; ++rr) {
                             const int r = r0 + rr;
-                            if (rv[u] && vec < V && ws[u][r] != 0.f)
+                            if (rv[u] && vec < V && ((msk[u] >> r) & 1u))
                                 v[u][e][rr] = ld_stream(
                                     reinterpret_cast<const uint4*>(a.o[r] + sb[u]) + vec);
                             else
@@ -140,7 +160,7 @@ __global__ void __launch_bounds__(kPullThreads) pull_combine_kernel(const PullAr
                     for (int e = 0; e < VPL; ++e)
 #pragma unroll
                         for (int rr = 0; rr < RB; ++rr) {
-                            const float wr = ws[u][r0 + rr];
+                            const float wr = wtab[wib][kk[u]][r0 + rr];
                             const uint32_t wd[4] = {v[u][e][rr].x, v[u][e][rr].y, v[u][e][rr].z,
                                                     v[u][e][rr].w};
 #pragma unroll

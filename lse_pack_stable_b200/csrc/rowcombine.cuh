@@ -16,10 +16,14 @@
 //     each rank's plane), forms each LSE, and computes M, the sum, LSE* and the
 //     W weights sequentially in rank order, all in registers.
 //   Phase B: G lanes cover one row's D elements with 16-byte vectors (VPL per
-//     lane), 32/G rows per step. The row's weights and addresses reach the
-//     group by warp shuffles from the lane that owns the row. Every rank's
-//     vector is loaded before any is used (U steps at once), accumulated in
-//     fp32 in rank order, rounded to the payload type and stored.
+//     lane), 32/G rows per step. The row's weights reach the group through a
+//     per-warp table in shared memory that phase A writes; its addresses and a
+//     mask of the ranks with nonzero weight come by warp shuffles from the
+//     lane that owns the row. (Shuffling all W weights to every lane held them
+//     twice in registers: on the 16-rank stress workload the table measured
+//     2 % faster.) Every rank's vector is loaded before any is used (U steps at
+//     once), accumulated in fp32 in rank order, rounded to the payload type
+//     and stored.
 // An invalid contribution (weight 0) is neither loaded nor added: its payload
 // is replaced by -0.0, which leaves the fp32 accumulator (started at -0.0)
 // unchanged bit for bit.
@@ -165,16 +169,31 @@ __device__ __forceinline__ void row_stats(const CombineArgs& a, int64_t q, bool 
     }
 }
 
+// Rows of one 16-byte vector per lane (D <= 256) keep four blocks resident: a
+// register budget of 128 per thread, which the 16-rank stress workload needs
+// for its loads in flight and which the compiler would exceed unbidden in
+// combine mode. Wider rows need more registers for their vectors.
+template <int VPL>
+constexpr int merge_min_blocks()
+{
+    return VPL == 1 ? 4 : 1;
+}
+
 template <typename P, int MODE, int WMAX, int G, int VPL, int U>
-__global__ void __launch_bounds__(kCombineThreads)
+__global__ void __launch_bounds__(kCombineThreads, merge_min_blocks<VPL>())
 rowcombine_kernel(const CombineArgs a)
 {
     constexpr int RPI = 32 / G;          // rows per step
     constexpr int STEPS = 32 / RPI;      // steps per chunk
-    constexpr int RB = WMAX < 16 ? WMAX : 16;   // ranks loaded at once
+    // ranks loaded at once: 16 vectors in flight per lane per batch
+    constexpr int RB = WMAX < 16 / VPL ? WMAX : 16 / VPL;
+    constexpr int WS = (WMAX + 3) / 4 * 4;
     static_assert(STEPS % U == 0, "U must divide the steps of a chunk");
+    // per-warp row table: the weights of the chunk's 32 rows
+    __shared__ __align__(16) float wtab[kCombineThreads / 32][32][WS];
 
     const int lane = threadIdx.x & 31;
+    const int wib = threadIdx.x >> 5;
     const int sub = lane / G;
     const int gl = lane % G;
     const int64_t warp = ((int64_t)blockIdx.x * kCombineThreads + threadIdx.x) >> 5;
@@ -199,29 +218,42 @@ rowcombine_kernel(const CombineArgs a)
         const int64_t q = c0 + lane;
         const bool qv = lane < cn;
         int64_t src_row, dst_row;
-        float lse[WMAX];
-        row_stats<MODE, WMAX>(a, q, qv, src_row, dst_row, lse);
+        uint32_t vmask = 0;               // bit r: contribution r has a nonzero weight
+        bool row_dead;
+        {
+            float lse[WMAX];
+            row_stats<MODE, WMAX>(a, q, qv, src_row, dst_row, lse);
+            float w[WS];
+            float L;
+            row_dead = !merge_weights(lse, w, L);
+            if (qv) st_stream(a.out_lse + dst_row, L);
+#pragma unroll
+            for (int r = 0; r < WMAX; ++r) vmask |= (w[r] != 0.f ? 1u : 0u) << r;
+            __syncwarp();                 // the previous chunk's table is read
+#pragma unroll
+            for (int r = 0; r < WS; r += 4)
+                *reinterpret_cast<float4*>(&wtab[wib][lane][r]) =
+                    make_float4(w[r], w[r + 1], w[r + 2], w[r + 3]);
+            __syncwarp();                 // the table is visible to the warp
+        }
 
-        float w[WMAX];
-        float L;
-        const bool row_dead = !merge_weights(lse, w, L);
-        if (qv) st_stream(a.out_lse + dst_row, L);
-
-        // ---------------- phase B: G lanes per row
+        // ---------------- phase B: G lanes per row; the row's weights come from
+        // the table, its addresses and valid-rank mask from the owning lane
 #pragma unroll 1
         for (int s0 = 0; s0 < STEPS; s0 += U) {
             int64_t sb[U], db[U];
             bool rv[U], dead[U];
-            float ws[U][WMAX];
+            uint32_t msk[U];
+            int kk[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int k = (s0 + u) * RPI + sub;
+                kk[u] = k;
                 sb[u] = __shfl_sync(kFull, src_row, k);
                 db[u] = __shfl_sync(kFull, dst_row, k);
                 dead[u] = __shfl_sync(kFull, (int)row_dead, k) != 0;
+                msk[u] = __shfl_sync(kFull, vmask, k);
                 rv[u] = k < cn;
-#pragma unroll
-                for (int r = 0; r < WMAX; ++r) ws[u][r] = __shfl_sync(kFull, w[r], k);
             }
             float acc[U][VPL][8];
 #pragma unroll
@@ -231,8 +263,8 @@ rowcombine_kernel(const CombineArgs a)
 #pragma unroll
                     for (int x = 0; x < 8; ++x) acc[u][e][x] = -0.f;
 
-#pragma unroll
-            for (int r0 = 0; r0 < WMAX; r0 += RB) {
+#pragma unroll 1
+            for (int r0 = 0; r0 < WMAX; r0 += RB) {   // one batch of ranks at a time
                 uint4 v[U][VPL][RB];
 #pragma unroll
                 for (int u = 0; u < U; ++u)
@@ -243,7 +275,7 @@ rowcombine_kernel(const CombineArgs a)
 #pragma unroll
                         for (int rr = 0; rr < RB; ++rr) {
                             const int r = r0 + rr;
-                            if (rv[u] && vec < V && ws[u][r] != 0.f)
+                            if (rv[u] && vec < V && ((msk[u] >> r) & 1u))
                                 v[u][e][rr] = ld_stream(base + (r * rank_stride >> 3));
                             else
                                 v[u][e][rr] = make_uint4(kNegZero2, kNegZero2, kNegZero2, kNegZero2);
@@ -255,7 +287,7 @@ rowcombine_kernel(const CombineArgs a)
                     for (int e = 0; e < VPL; ++e)
 #pragma unroll
                         for (int rr = 0; rr < RB; ++rr) {
-                            const float wr = ws[u][r0 + rr];
+                            const float wr = wtab[wib][kk[u]][r0 + rr];
                             const uint32_t wd[4] = {v[u][e][rr].x, v[u][e][rr].y, v[u][e][rr].z,
                                                     v[u][e][rr].w};
 #pragma unroll
