@@ -198,8 +198,9 @@ def recorded_traffic(config: str):
     return int(tr.group(1))
 
 
-def merge_kernel_name(W: int) -> str:
-    return ("rowcombine_kernel (register-staged, fused mode)" if W > 8
+def merge_kernel_name(W: int, D: int) -> str:
+    """The merge kernel the library launches for W ranks and head dim D."""
+    return ("rowcombine_kernel (register-staged, fused mode)" if W > 8 or D > 256
             else "rowcombine_async_kernel (shared-memory-staged, fused mode)")
 
 
@@ -534,7 +535,7 @@ def measure_workload(cp, wl, dev, stream, args, world, barrier, peak, peak_kind,
     overlapped = bytes_per_call / (ms_per_step * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": recorded_traffic(wl.name),
-                "peak_source": peak_source(peak_kind), "kernel": merge_kernel_name(wl.W),
+                "peak_source": peak_source(peak_kind), "kernel": merge_kernel_name(wl.W, wl.D),
                 "algorithmic_bytes_per_launch": bytes_per_call,
                 "us_per_launch": round(med_launch * 1e3, 3),
                 "us_per_launch_p10_p50_p90": [round(1e3 * pct(launch_ms, q), 3)

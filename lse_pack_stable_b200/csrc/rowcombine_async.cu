@@ -36,14 +36,20 @@ cudaError_t launch_async_inst(const CombineArgs& a, cudaStream_t s)
     return launch_pdl(kern, (unsigned)blocks, kAsyncThreads, smem, s, a);
 }
 
-// Shared-memory staging for up to 8 ranks; register staging from 16 ranks on,
-// where one step of every rank is 8 KB or more per warp and the register-staged
-// kernel measured faster (W=16, D=128: 2.95 ms against 3.3-4.4 ms).
+// Shared-memory staging for up to 8 ranks with rows of one 16-byte vector per
+// lane (D <= 256); register staging otherwise. From 16 ranks on, one step of
+// every rank is 8 KB or more per warp and the ring leaves too few warps
+// resident (stress, W=16 D=128: 2.95 ms against 3.3-4.4 ms). For wider rows the
+// register path with its per-warp weight table keeps 16 vectors per lane in
+// flight and measured faster (mla, W=8 D=512: 1405 against 1516 us); for
+// D = 128 at 4 and 8 ranks the ring stays ahead (ulysses: 572 against 580 us).
 template <typename P, int MODE, int WMAX, int G, int VPL>
 cudaError_t launch_staged(const CombineArgs& a, cudaStream_t s)
 {
-    if (WMAX >= 16) return launch_rowcombine_inst<P, MODE, WMAX, G, VPL>(a, s);
-    return launch_async_inst<P, MODE, WMAX, G, VPL>(a, s);
+    if constexpr (WMAX >= 16 || VPL >= 2)
+        return launch_rowcombine_inst<P, MODE, WMAX, G, VPL>(a, s);
+    else
+        return launch_async_inst<P, MODE, WMAX, G, VPL>(a, s);
 }
 
 template <typename P, int MODE, int WMAX>

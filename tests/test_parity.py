@@ -44,9 +44,11 @@ CASES = [
         last_token_invalid=True),
     _wl("w7_d40", 7, 19, 14, 40, dtype="fp16", p_invalid=0.2),
     _wl("w4_d256_many_invalid", 4, 33, 8, 256, p_invalid=0.6),
-    # the largest shared-memory ring (205 KB per block, one block per SM) and the
-    # widest register-staged row: D = 1024 at W = 8 and at W = 32
+    # the widest register-staged rows (four 16-byte vectors per lane, ranks in
+    # batches of four): D = 1024 at W = 8 and at W = 32; and the largest
+    # shared-memory ring, D = 256 at W = 8 (one vector per lane, 32 lanes)
     _wl("w8_d1024_ring_max", 8, 5, 16, 1024, p_invalid=0.1),
+    _wl("w8_d256_ring", 8, 9, 16, 256, p_invalid=0.1),
     _wl("w32_d1024_max", 32, 2, 32, 1024, p_invalid=0.1),
 ]
 IDS = [c.name for c in CASES]

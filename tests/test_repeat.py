@@ -1,8 +1,10 @@
 """Back-to-back launches give the same bits.
 
-The merge kernels stream rows through rings of shared-memory stages filled
-asynchronously; a mistake in the ring bookkeeping (a slot refilled before it
-is read, a wait one group short) shows up as a race that depends on timing,
+The shared-memory-staged merge streams rows through rings of stages filled
+asynchronously, and the register-staged merge passes each chunk's weights
+through a per-warp table; a mistake in that bookkeeping (a slot or a table
+refilled before it is read, a wait one group short) shows up as a race that
+depends on timing,
 so one passing run proves little. Each case here launches the same call many
 times, with other work queued in between, and requires every result to be
 bit-identical to the first.
