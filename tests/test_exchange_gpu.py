@@ -90,6 +90,26 @@ def test_combine_rank_is_a_destination_of_the_combine(wl, orc):
                        wl.W)
 
 
+@pytest.mark.parametrize("wl", [w for w in TOKEN_CASES if w.T % w.W == 0][:6],
+                         ids=[w.name for w in TOKEN_CASES if w.T % w.W == 0][:6])
+def test_combine_rank_on_token_chunks(wl):
+    """The token-chunk packet: destination j's received [W, T/W, H, D] is
+    combined with T/W as T and H as Hc, and equals destination j of the
+    W-rank combine and of the token-chunk fused call."""
+    (o, m, s), (do, dm, ds) = _dev(wl)
+    pkt, pl = cp.cp_pack_lse(do, dm, ds, scatter_dim=0)
+    ro, rl = cp.cp_a2a_local_permute(pkt, wl.W), cp.cp_a2a_local_permute(pl, wl.W)
+    out, out_lse = cp.cp_lse_combine(ro, rl)
+    fo, fl = cp.cp_pack_permute_combine_fused(do, dm, ds, scatter_dim=0)
+    for j in range(wl.W):
+        oj, lj = cp.cp_lse_combine_rank(ro[j], rl[j])
+        torch.cuda.synchronize()
+        assert torch.equal(oj.view(torch.int16), out[j].view(torch.int16)), "destination %d" % j
+        assert torch.equal(lj.view(torch.int32), out_lse[j].view(torch.int32))
+        assert torch.equal(oj.view(torch.int16), fo[j].view(torch.int16))
+        assert torch.equal(lj.view(torch.int32), fl[j].view(torch.int32))
+
+
 def _separate_planes(do, dm, ds, strided):
     """W separately allocated planes per tensor (optionally strided views)."""
     os_, ms, ss = [], [], []
