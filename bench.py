@@ -633,7 +633,7 @@ def run_ours(args):
 # --------------------------------------------------------------------------------------------
 # N > 1 GPUs: the exchange across real ranks
 
-NVLINK_PEER_GBS = 770.0        # measured peer copy per direction on this machine's B200s
+NVLINK_PEER_GBS = 770.0        # measured B200 peer copy over NVLink 5, per direction per GPU
 
 
 def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
@@ -728,7 +728,7 @@ def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
         "roofline": {"bound": "nvlink", "achieved": round(achieved, 2), "peak": NVLINK_PEER_GBS,
                      "unit": "GB/s", "frac": round(achieved / NVLINK_PEER_GBS, 4),
                      "traffic": None, "kernel": "pull_combine_kernel (plain loads over NVLink)",
-                     "peak_source": "measured peer copy per direction on this pool (770 GB/s)",
+                     "peak_source": "measured B200 peer copy per direction (770 GB/s)",
                      "nvlink_bytes_per_rank_per_call": remote},
         "clocks": clocks.summary(), "gpu_launches": K,
         "e2e": {"value": round(bytes_per_call * ke / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
