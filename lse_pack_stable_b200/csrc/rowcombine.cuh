@@ -63,7 +63,7 @@ struct ChunkPlan {
     int64_t last_base;        // first row of the last, partial round
     int64_t last_rows;        // rows per warp in the last round (<= 32)
 
-    __device__ __forceinline__ ChunkPlan(int64_t rows_, int64_t warp_, int64_t nwarps_)
+    __host__ __device__ __forceinline__ ChunkPlan(int64_t rows_, int64_t warp_, int64_t nwarps_)
         : rows(rows_), warp(warp_), nwarps(nwarps_)
     {
         full = rows / (32 * nwarps);
@@ -72,13 +72,13 @@ struct ChunkPlan {
     }
 
     // chunks of this warp
-    __device__ __forceinline__ int64_t count() const
+    __host__ __device__ __forceinline__ int64_t count() const
     {
         return full + (last_base + warp * last_rows < rows ? 1 : 0);
     }
 
     // chunk i of this warp: its first row and its row count (1..32)
-    __device__ __forceinline__ void chunk(int64_t i, int64_t& start, int& n) const
+    __host__ __device__ __forceinline__ void chunk(int64_t i, int64_t& start, int& n) const
     {
         if (i < full) {
             start = (warp + i * nwarps) * 32;
