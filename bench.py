@@ -692,6 +692,10 @@ def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
     pull_ms = time_back_to_back(lambda i: pull(out_p, lse_p), stream, K, Wm, barrier)
     a2a_ms = time_back_to_back(lambda i: a2a(pull.o, pull.smax, pull.ssum, out_a, lse_a), stream,
                                K, Wm, barrier)
+    # per call, the slowest rank (the FastVideo page's rank-max p50/p95)
+    pull_calls = rank_max_calls(lambda i: pull(out_p, lse_p), stream, K, world, dev)
+    a2a_calls = rank_max_calls(lambda i: a2a(pull.o, pull.smax, pull.ssum, out_a, lse_a), stream,
+                               K, world, dev)
     clocks.stop()
     pull_ms, a2a_ms = reduce_max([pull_ms, a2a_ms], world, dev)
     bytes_per_call = wl.fused_bytes()                 # every rank's reads and writes together
@@ -735,6 +739,8 @@ def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
                 "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world,
                 "ms_per_step": round(e2e_ms / ke, 4), "steps": ke},
         "exchange": {"pull_equals_a2a": bool(same.item() == 1.0),
+                     "pull_rank_max_us_p50_p95": [round(1e3 * pct(pull_calls, q), 3) for q in (50, 95)],
+                     "a2a_rank_max_us_p50_p95": [round(1e3 * pct(a2a_calls, q), 3) for q in (50, 95)],
                      "a2a_us_per_call": round(a2a_ms / K * 1e3, 3),
                      "a2a_GB/s": round(bytes_per_call * K / (a2a_ms * 1e-3) / 1e9, 2),
                      "a2a_path": "cp_pack_lse_rank -> NCCL all-to-all x2 -> cp_lse_combine_rank",
@@ -748,6 +754,26 @@ def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
     torch.cuda.synchronize()
     pull.close()
     return 0
+
+
+def rank_max_calls(fn, stream, reps, world, dev):
+    """Each of `reps` calls timed on its own (events around it, a barrier of the
+    group before it), then, call by call, the slowest rank's time (ms)."""
+    import torch
+    import torch.distributed as dist
+    for i in range(3):
+        fn(i)
+    torch.cuda.synchronize()
+    ms = []
+    for i in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        a.record(stream)
+        fn(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b))
+    return reduce_max(ms, world, dev)
 
 
 def all_to_all_4d_nccl(x, scatter_dim, gather_dim, world, out_shape):

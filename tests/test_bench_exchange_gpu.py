@@ -39,5 +39,7 @@ def test_bench_exchange_two_ranks_on_one_gpu(config, extra):
     assert rec["n_gpus"] == 2 and rec["config"]["parallelism"] == "dcp2"
     assert rec["exchange"]["pull_equals_a2a"] is True
     assert rec["value"] > 0 and rec["roofline"]["bound"] == "nvlink"
+    p50, p95 = rec["exchange"]["pull_rank_max_us_p50_p95"]
+    assert 0 < p50 <= p95
     if config == "ulysses":
         assert rec["ulysses_exchange"]["pull_equals_nccl"] is True
