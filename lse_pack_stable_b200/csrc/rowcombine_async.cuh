@@ -15,7 +15,12 @@
 // Work: warp w owns chunks w, w + nwarps, ... of 32 output rows; a chunk has
 // STEPS = G steps of RPI = 32/G rows. A "group" is one step of one chunk;
 // group number n of the warp is chunk n / STEPS, step n % STEPS (compile-time
-// divisors). Group n lands in ring slot n % NST. The first group of a chunk
+// divisors), and that step covers rows ((n + w) mod STEPS) * RPI .. of the
+// chunk: every warp starts its chunks at a different step, so that warps in
+// lockstep do not all touch the same offset of their chunks at once (measured:
+// 2-3 % on a 4-rank decode merge, 1-1.5 % on an 8-rank one; the register-staged
+// kernel of rowcombine.cuh gained nothing from it and keeps step order).
+// Group n lands in ring slot n % NST. The first group of a chunk
 // also brings the chunk's statistics (lane = row) into statistics slot
 // chunk % NSTAT, where NSTAT = (NST-1)/STEPS + 1 guarantees the slot was read
 // (phase A of an older chunk) before it is refilled NST-1 groups ahead.
@@ -124,6 +129,13 @@ rowcombine_async_kernel(const CombineArgs a)
     const int64_t nwarps = ((int64_t)gridDim.x * kAsyncThreads) >> 5;
     const ChunkPlan plan(a.rows, warp, nwarps);
     const int64_t ngroups = plan.count() * STEPS;
+    // Each warp walks the steps of its chunks starting at step warp mod STEPS.
+    // Warps run nearly in lockstep, and chunks start on 32-row boundaries, so
+    // without this every warp would be reading (and writing) the same offset
+    // within its chunk at the same moment; rotated, the accesses in flight
+    // spread over STEPS offsets. Each row's arithmetic is unchanged.
+    static_assert((STEPS & (STEPS - 1)) == 0, "steps per chunk must be a power of two");
+    const int rot = (int)(warp & (STEPS - 1));
 
     // Programmatic dependent launch: the next kernel in the stream may be
     // scheduled now, and this one reads nothing until the previous kernel in
@@ -189,7 +201,7 @@ rowcombine_async_kernel(const CombineArgs a)
                     }
                 }
             }
-            const int kq = st_i * RPI + sub;                 // row of the chunk
+            const int kq = ((st_i + rot) & (STEPS - 1)) * RPI + sub;   // row of the chunk
             if (kq < cn_i) {
                 const int64_t off = lin_i ? chunk_src + kq * V : row_src(c0_i + kq);
                 const uint4* base = src16 + off + gl;
@@ -268,7 +280,7 @@ rowcombine_async_kernel(const CombineArgs a)
             __syncwarp();                                   // the table is visible to the warp
         }
         // ---------------- phase B: this step's RPI rows, G lanes per row
-        const int k = step * RPI + sub;                     // row of the chunk
+        const int k = ((step + rot) & (STEPS - 1)) * RPI + sub;     // row of the chunk
         if (k < cn) {
             int64_t db = dtab[k];
             const bool dead = db < 0;
