@@ -75,10 +75,10 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const PackArgs a)
             src_row = r * a.so_r + t * a.so_t + h * a.so_h;
             if (FROM_LSE) {
                 // legacy: the materialized LSE moves into the packet layout
-                st_stream(a.pkt_lse + dst_row, ld_stream(a.lse + r * a.sm_r + t * a.sm_t + h * a.sm_h));
+                st_stream(a.pkt_lse + dst_row, ld_ro(a.lse + r * a.sm_r + t * a.sm_t + h * a.sm_h));
             } else {
-                const float m = ld_stream(a.smax + r * a.sm_r + t * a.sm_t + h * a.sm_h);
-                const float s = ld_stream(a.ssum + r * a.ss_r + t * a.ss_t + h * a.ss_h);
+                const float m = ld_ro(a.smax + r * a.sm_r + t * a.sm_t + h * a.sm_h);
+                const float s = ld_ro(a.ssum + r * a.ss_r + t * a.ss_t + h * a.ss_h);
                 const bool ok = isfinite(m) && isfinite(s) && s > 0.f;
                 st_stream(a.pkt_lse + dst_row, ok ? m + logf(s) : -INFINITY);
             }
@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const PackArgs a)
                 for (int e = 0; e < VPL; ++e) {
                     const int vec = gl + e * G;
                     if (rv[u] && vec < V)
-                        v[u][e] = ld_stream(reinterpret_cast<const uint4*>(a.o + sb[u]) + vec);
+                        v[u][e] = ld_ro(reinterpret_cast<const uint4*>(a.o + sb[u]) + vec);
                 }
             }
 #pragma unroll
@@ -169,7 +169,7 @@ pack_block_kernel(const PackArgs a, int64_t pay_cols)
             if (k < nvec) {
                 int64_t t, off;
                 divmod_pack(k, HcV, t, off);
-                v[u] = ld_stream(src + t * st8 + off);
+                v[u] = ld_ro(src + t * st8 + off);
             }
         }
 #pragma unroll
@@ -188,10 +188,10 @@ pack_block_kernel(const PackArgs a, int64_t pay_cols)
             const int64_t h = (int64_t)j * a.Hc + hc;
             float lv;
             if (FROM_LSE) {
-                lv = ld_stream(a.lse + r * a.sm_r + t * a.sm_t + h * a.sm_h);
+                lv = ld_ro(a.lse + r * a.sm_r + t * a.sm_t + h * a.sm_h);
             } else {
-                const float m = ld_stream(a.smax + r * a.sm_r + t * a.sm_t + h * a.sm_h);
-                const float sv = ld_stream(a.ssum + r * a.ss_r + t * a.ss_t + h * a.ss_h);
+                const float m = ld_ro(a.smax + r * a.sm_r + t * a.sm_t + h * a.sm_h);
+                const float sv = ld_ro(a.ssum + r * a.ss_r + t * a.ss_t + h * a.ss_h);
                 const bool ok = isfinite(m) && isfinite(sv) && sv > 0.f;
                 lv = ok ? m + logf(sv) : -INFINITY;
             }
@@ -243,8 +243,8 @@ __global__ void __launch_bounds__(kMatThreads) lse_materialize_kernel(const Pack
         int64_t r, rem, t, h;
         divmod_pack(q, TH, r, rem);
         divmod_pack(rem, (int64_t)a.H, t, h);
-        const float m = ld_stream(a.smax + r * a.sm_r + t * a.sm_t + h * a.sm_h);
-        const float sv = ld_stream(a.ssum + r * a.ss_r + t * a.ss_t + h * a.ss_h);
+        const float m = ld_ro(a.smax + r * a.sm_r + t * a.sm_t + h * a.sm_h);
+        const float sv = ld_ro(a.ssum + r * a.ss_r + t * a.ss_t + h * a.ss_h);
         const bool ok = isfinite(m) && isfinite(sv) && sv > 0.f;
         st_stream(lse + q, ok ? m + logf(sv) : -INFINITY);
     }

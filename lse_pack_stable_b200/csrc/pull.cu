@@ -91,8 +91,8 @@ pull_combine_kernel(const PullArgs a)
             for (int r = 0; r < WMAX; ++r) {
                 float m = -INFINITY, sm = 0.f;
                 if (qv && r < a.W) {
-                    m = ld_stream(a.smax[r] + mo);
-                    sm = ld_stream(a.ssum[r] + so);
+                    m = ld_ro(a.smax[r] + mo);
+                    sm = ld_ro(a.ssum[r] + so);
                 }
                 // invalid statistic: non-finite max, non-finite sum, or sum <= 0
                 const bool ok = isfinite(m) && isfinite(sm) && sm > 0.f;
@@ -148,7 +148,7 @@ pull_combine_kernel(const PullArgs a)
                         for (int rr = 0; rr < RB; ++rr) {
                             const int r = r0 + rr;
                             if (rv[u] && vec < V && ((msk[u] >> r) & 1u))
-                                v[u][e][rr] = ld_stream(
+                                v[u][e][rr] = ld_ro(
                                     reinterpret_cast<const uint4*>(a.o[r] + sb[u]) + vec);
                             else
                                 v[u][e][rr] = make_uint4(kNegZero2, kNegZero2, kNegZero2, kNegZero2);

@@ -139,8 +139,8 @@ __device__ __forceinline__ void row_stats(const CombineArgs& a, int64_t q, bool 
 #pragma unroll
         for (int r = 0; r < WMAX; ++r) {
             if (qv && r < a.W) {
-                m[r] = ld_stream(pm + r * a.sm_r);
-                s[r] = ld_stream(ps + r * a.ss_r);
+                m[r] = ld_ro(pm + r * a.sm_r);
+                s[r] = ld_ro(ps + r * a.ss_r);
             } else {
                 m[r] = -INFINITY;
                 s[r] = 0.f;
@@ -163,7 +163,7 @@ __device__ __forceinline__ void row_stats(const CombineArgs& a, int64_t q, bool 
         const float* pl = a.lse + j * a.W * a.N + n;
 #pragma unroll
         for (int r = 0; r < WMAX; ++r) {
-            float x = (qv && r < a.W) ? ld_stream(pl + r * a.N) : -INFINITY;
+            float x = (qv && r < a.W) ? ld_ro(pl + r * a.N) : -INFINITY;
             lse[r] = x > -INFINITY ? x : -INFINITY;   // NaN counts as invalid
         }
     }
@@ -276,7 +276,7 @@ rowcombine_kernel(const CombineArgs a)
                         for (int rr = 0; rr < RB; ++rr) {
                             const int r = r0 + rr;
                             if (rv[u] && vec < V && ((msk[u] >> r) & 1u))
-                                v[u][e][rr] = ld_stream(base + (r * rank_stride >> 3));
+                                v[u][e][rr] = ld_ro(base + (r * rank_stride >> 3));
                             else
                                 v[u][e][rr] = make_uint4(kNegZero2, kNegZero2, kNegZero2, kNegZero2);
                         }
