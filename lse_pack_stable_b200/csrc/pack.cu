@@ -136,12 +136,14 @@ cudaError_t launch_pack_inst(const PackArgs& a, cudaStream_t s)
     return cudaGetLastError();
 }
 
-// Head-chunk pack of rank rows that are back to back (so_h == D), one packet
-// block (r, j) per grid row: the block is T rows of Hc*D contiguous elements,
-// row t copied from source (r, t) at head j*Hc. Each thread moves U 16-byte
-// vectors (all loads in flight before the first store) and the grid covers
-// the block once, so blocks retire and start continuously. The last grid
-// columns form (or, legacy, move) the block's T*Hc LSE values.
+// Head-chunk pack of rank rows that are back to back (so_h == D). Packet
+// block (r, j) is T rows of Hc*D contiguous elements, row t copied from source
+// (r, t) at head j*Hc. Each thread moves U 16-byte vectors (all loads in
+// flight before the first store) and the grid covers every block once, so
+// blocks retire and start continuously; grid.y is the source rank, grid.x
+// enumerates (column, destination) with the destination fastest. Columns
+// below lse_cols form (or, legacy, move) the block's T*Hc LSE values, the
+// rest copy the payload.
 #ifndef CPLSE_PACK_U
 #define CPLSE_PACK_U 8
 #endif
@@ -150,18 +152,26 @@ constexpr int kBlockU = CPLSE_PACK_U;
 
 template <bool FROM_LSE>
 __global__ void __launch_bounds__(kBlockThreads)
-pack_block_kernel(const PackArgs a, int64_t pay_cols)
+pack_block_kernel(const PackArgs a, int64_t pay_cols, int64_t lse_cols)
 {
-    const int rj = blockIdx.y;                              // (source r, destination j)
-    const int r = rj / a.W, j = rj - r * a.W;
+    // Grid order: the destination j varies fastest, so that the blocks running
+    // at the same time copy every head chunk of the same source rows, i.e. read
+    // whole token rows between them instead of one Hc*D piece of each row
+    // (stress 5712 -> 5386 us, mla 2632 -> 2526 us). The LSE columns come
+    // first, so that their latency overlaps the payload copy.
+    const int j = (int)(blockIdx.x % (unsigned)a.W);
+    const int r = blockIdx.y;                               // source rank
+    const int rj = r * a.W + j;                             // packet block (r, j)
+    int64_t bx = blockIdx.x / (unsigned)a.W;
+    bx = bx < lse_cols ? pay_cols + bx : bx - lse_cols;     // payload columns: bx < pay_cols
     const int64_t HcV = (int64_t)a.Hc * (a.D >> 3);        // vectors per packet row
     const int64_t block_rows = a.T * a.Hc;
-    if ((int64_t)blockIdx.x < pay_cols) {
+    if (bx < pay_cols) {
         const int64_t nvec = a.T * HcV;
         const uint4* src = reinterpret_cast<const uint4*>(a.o + r * a.so_r + (int64_t)j * a.Hc * a.D);
         uint4* dst = reinterpret_cast<uint4*>(a.pkt_o) + (int64_t)rj * nvec;
         const int64_t st8 = a.so_t >> 3;
-        const int64_t base = (int64_t)blockIdx.x * kBlockThreads * kBlockU + threadIdx.x;
+        const int64_t base = bx * kBlockThreads * kBlockU + threadIdx.x;
         uint4 v[kBlockU];
 #pragma unroll
         for (int u = 0; u < kBlockU; ++u) {
@@ -178,7 +188,7 @@ pack_block_kernel(const PackArgs a, int64_t pay_cols)
             if (k < nvec) st_stream(dst + k, v[u]);
         }
     } else {
-        const int64_t base = ((int64_t)blockIdx.x - pay_cols) * kBlockThreads * 4 + threadIdx.x;
+        const int64_t base = (bx - pay_cols) * kBlockThreads * 4 + threadIdx.x;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int64_t k = base + (int64_t)u * kBlockThreads;
@@ -206,9 +216,9 @@ cudaError_t launch_pack_blocks(const PackArgs& a, cudaStream_t s)
     const int64_t HcV = (int64_t)a.Hc * (a.D >> 3);
     const int64_t pay_cols = (a.T * HcV + kBlockThreads * kBlockU - 1) / (kBlockThreads * kBlockU);
     const int64_t lse_cols = (a.T * a.Hc + kBlockThreads * 4 - 1) / (kBlockThreads * 4);
-    if (pay_cols + lse_cols > 0x7fffffff) return cudaErrorInvalidConfiguration;
-    dim3 grid((unsigned)(pay_cols + lse_cols), (unsigned)(a.nsrc * a.W));
-    pack_block_kernel<FROM_LSE><<<grid, kBlockThreads, 0, s>>>(a, pay_cols);
+    if ((pay_cols + lse_cols) * a.W > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    dim3 grid((unsigned)((pay_cols + lse_cols) * a.W), (unsigned)a.nsrc);
+    pack_block_kernel<FROM_LSE><<<grid, kBlockThreads, 0, s>>>(a, pay_cols, lse_cols);
     return cudaGetLastError();
 }
 
