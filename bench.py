@@ -1001,6 +1001,15 @@ def measure_breakdown(cp, wl, sets, stream, dev, peak):
     def pack(i):
         cp.cp_pack_lse(*sets[i % n][:3], pkt_o=pk[i % nb][0], pkt_lse=pk[i % nb][1], stream=stream)
     rec("pack", pack, wl.pack_bytes())
+    if T % W == 0:
+        # the token-chunk packet (scatter_dim = 0) in the same buffers, viewed [W][W][T/W][H]
+        tpk = [(p[0].view(W, W, T // W, H, D), p[1].view(W, W, T // W, H)) for p in pk]
+
+        def pack_tokens(i):
+            cp.cp_pack_lse(*sets[i % n][:3], scatter_dim=0, pkt_o=tpk[i % nb][0],
+                           pkt_lse=tpk[i % nb][1], stream=stream)
+        rec("pack_token_chunks", pack_tokens, wl.pack_bytes())
+        del tpk
     rows = W * T * H
     # the Before pipeline of the DCP pull request: materialize LSE, then pack from it
     lse_buf = torch.empty((W, T, H), dtype=torch.float32, device=dev)

@@ -136,19 +136,30 @@ cudaError_t launch_pack_inst(const PackArgs& a, cudaStream_t s)
     return cudaGetLastError();
 }
 
-// Head-chunk pack of rank rows that are back to back (so_h == D). Packet
-// block (r, j) is T rows of Hc*D contiguous elements, row t copied from source
-// (r, t) at head j*Hc. Each thread moves U 16-byte vectors (all loads in
-// flight before the first store) and the grid covers every block once, so
-// blocks retire and start continuously; grid.y is the source rank, grid.x
-// enumerates (column, destination) with the destination fastest. Columns
-// below lse_cols form (or, legacy, move) the block's T*Hc LSE values, the
-// rest copy the payload.
+// Block-copy pack of rank rows that are back to back (so_h == D). Packet block
+// (r, j) is NB rows of RE contiguous elements:
+//   head chunks  (scatter_dim 1): NB = T rows of Hc*D, row t read from source
+//                (r, t) at head j*Hc;
+//   token chunks (scatter_dim 0): NB = T/W rows of H*D, row tc read from source
+//                (r, j*T/W + tc), i.e. the whole block is one run of token rows.
+// Each thread moves U 16-byte vectors (all loads in flight before the first
+// store) and the grid covers every block once, so blocks retire and start
+// continuously; grid.y is the source rank, grid.x enumerates (column,
+// destination) with the destination fastest. Columns below lse_cols form (or,
+// legacy, move) the block's LSE values, the rest copy the payload.
 #ifndef CPLSE_PACK_U
 #define CPLSE_PACK_U 8
 #endif
 constexpr int kBlockThreads = 256;
 constexpr int kBlockU = CPLSE_PACK_U;
+
+// rows per packet block and 16-byte vectors per packet row
+__host__ __device__ __forceinline__ void pack_block_shape(const PackArgs& a, int64_t& nb, int64_t& rv)
+{
+    const bool tok = a.scatter_dim == 0;
+    nb = tok ? a.Tc : a.T;
+    rv = ((int64_t)(tok ? a.H : a.Hc) * a.D) >> 3;
+}
 
 template <bool FROM_LSE>
 __global__ void __launch_bounds__(kBlockThreads)
@@ -164,11 +175,13 @@ pack_block_kernel(const PackArgs a, int64_t pay_cols, int64_t lse_cols)
     const int rj = r * a.W + j;                             // packet block (r, j)
     int64_t bx = blockIdx.x / (unsigned)a.W;
     bx = bx < lse_cols ? pay_cols + bx : bx - lse_cols;     // payload columns: bx < pay_cols
-    const int64_t HcV = (int64_t)a.Hc * (a.D >> 3);        // vectors per packet row
-    const int64_t block_rows = a.T * a.Hc;
+    const bool tok = a.scatter_dim == 0;
+    int64_t nb, rv;
+    pack_block_shape(a, nb, rv);
     if (bx < pay_cols) {
-        const int64_t nvec = a.T * HcV;
-        const uint4* src = reinterpret_cast<const uint4*>(a.o + r * a.so_r + (int64_t)j * a.Hc * a.D);
+        const int64_t nvec = nb * rv;
+        const int64_t first = tok ? (int64_t)j * a.Tc * a.so_t : (int64_t)j * a.Hc * a.D;
+        const uint4* src = reinterpret_cast<const uint4*>(a.o + r * a.so_r + first);
         uint4* dst = reinterpret_cast<uint4*>(a.pkt_o) + (int64_t)rj * nvec;
         const int64_t st8 = a.so_t >> 3;
         const int64_t base = bx * kBlockThreads * kBlockU + threadIdx.x;
@@ -178,7 +191,7 @@ pack_block_kernel(const PackArgs a, int64_t pay_cols, int64_t lse_cols)
             const int64_t k = base + (int64_t)u * kBlockThreads;
             if (k < nvec) {
                 int64_t t, off;
-                divmod_pack(k, HcV, t, off);
+                divmod_pack(k, rv, t, off);
                 v[u] = ld_ro(src + t * st8 + off);
             }
         }
@@ -188,14 +201,18 @@ pack_block_kernel(const PackArgs a, int64_t pay_cols, int64_t lse_cols)
             if (k < nvec) st_stream(dst + k, v[u]);
         }
     } else {
+        // packet LSE k of block (r, j): row k / L, column k % L, L = H (tokens) or Hc (heads)
+        const int64_t L = tok ? a.H : a.Hc;
+        const int64_t block_rows = nb * L;
         const int64_t base = (bx - pay_cols) * kBlockThreads * 4 + threadIdx.x;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int64_t k = base + (int64_t)u * kBlockThreads;
             if (k >= block_rows) break;
-            int64_t t, hc;
-            divmod_pack(k, (int64_t)a.Hc, t, hc);
-            const int64_t h = (int64_t)j * a.Hc + hc;
+            int64_t row, col;
+            divmod_pack(k, L, row, col);
+            const int64_t t = tok ? (int64_t)j * a.Tc + row : row;
+            const int64_t h = tok ? col : (int64_t)j * a.Hc + col;
             float lv;
             if (FROM_LSE) {
                 lv = ld_ro(a.lse + r * a.sm_r + t * a.sm_t + h * a.sm_h);
@@ -213,9 +230,11 @@ pack_block_kernel(const PackArgs a, int64_t pay_cols, int64_t lse_cols)
 template <bool FROM_LSE>
 cudaError_t launch_pack_blocks(const PackArgs& a, cudaStream_t s)
 {
-    const int64_t HcV = (int64_t)a.Hc * (a.D >> 3);
-    const int64_t pay_cols = (a.T * HcV + kBlockThreads * kBlockU - 1) / (kBlockThreads * kBlockU);
-    const int64_t lse_cols = (a.T * a.Hc + kBlockThreads * 4 - 1) / (kBlockThreads * 4);
+    int64_t nb, rv;
+    pack_block_shape(a, nb, rv);
+    const int64_t L = a.scatter_dim == 0 ? a.H : a.Hc;
+    const int64_t pay_cols = (nb * rv + kBlockThreads * kBlockU - 1) / (kBlockThreads * kBlockU);
+    const int64_t lse_cols = (nb * L + kBlockThreads * 4 - 1) / (kBlockThreads * 4);
     if ((pay_cols + lse_cols) * a.W > 0x7fffffff) return cudaErrorInvalidConfiguration;
     dim3 grid((unsigned)((pay_cols + lse_cols) * a.W), (unsigned)a.nsrc);
     pack_block_kernel<FROM_LSE><<<grid, kBlockThreads, 0, s>>>(a, pay_cols, lse_cols);
@@ -225,8 +244,8 @@ cudaError_t launch_pack_blocks(const PackArgs& a, cudaStream_t s)
 template <bool FROM_LSE>
 cudaError_t launch_pack_l(const PackArgs& a, cudaStream_t s)
 {
-    // head chunks of back-to-back rows: chunk copies; anything else: row by row
-    if (a.scatter_dim == 1 && a.so_h == a.D) return launch_pack_blocks<FROM_LSE>(a, s);
+    // back-to-back rows: block copies (head or token chunks); anything else: row by row
+    if (a.so_h == a.D) return launch_pack_blocks<FROM_LSE>(a, s);
     const RowShape rs = row_shape(a.D);
     switch (rs.G * 10 + rs.VPL) {
     case 41: return launch_pack_inst<4, 1, FROM_LSE>(a, s);
