@@ -7,12 +7,12 @@
 // tensor; the rule for invalid statistics) and "How was this patch tested?"
 // (scatter_dim 0 and 1, non-contiguous output/max/sum strides).
 //
-// Two kernels. Head chunks with back-to-back rows take the 2-D block copy
-// further down. Everything else takes the row kernel: a warp owns chunks of 32
-// consecutive source rows (r, t, h) in input order. Phase A: lane i forms the LSE of row i (coalesced max/sum
-// loads) and writes it to the LSE region. Phase B: G lanes copy one row's D
-// elements with 16-byte vectors; U steps of loads are in flight before the
-// first store.
+// Two kernels. Back-to-back rows (so_h == D), head or token chunks, take the
+// 2-D block copy further down. Everything else takes the row kernel: a warp
+// owns chunks of 32 consecutive source rows (r, t, h) in input order. Phase A:
+// lane i forms the LSE of row i (coalesced max/sum loads) and writes it to the
+// LSE region. Phase B: G lanes copy one row's D elements with 16-byte vectors;
+// U steps of loads are in flight before the first store.
 #include <math.h>
 
 #include "common.cuh"
