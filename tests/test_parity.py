@@ -154,6 +154,35 @@ def test_pack_strided_inputs(orc):
     assert torch.equal(cl.view(torch.int32), fl.view(torch.int32))
 
 
+@pytest.mark.parametrize("scatter_dim", [1, 0])
+def test_pack_block_copy_padded_token_stride(scatter_dim, orc):
+    """Heads back to back within a token (so_h == D), gaps between tokens and
+    between ranks: the block-copy pack for head and for token chunks, its
+    legacy twin, and the per-rank pack of one such plane, against the oracle."""
+    wl = _wl("padded_tokens", 4, 20, 8, 64, p_invalid=0.05)
+    o, m, s = synth.full_inputs(wl)
+    W, T, H, D = o.shape
+    row = H * D + 64                                   # token stride: 64 elements of padding
+    big = torch.zeros((W + 1) * (T + 3) * row, dtype=torch.bfloat16, device="cuda")
+    ov = torch.as_strided(big, (W, T, H, D), ((T + 3) * row, row, D, 1), storage_offset=row + 8)
+    ov.copy_(dev_payload(o, "bf16"))
+    assert ov.stride(2) == D and ov.stride(1) != H * D
+    dm, ds = dev_f32(m), dev_f32(s)
+    pkt, pl = cp.cp_pack_lse(ov, dm, ds, scatter_dim=scatter_dim)
+    lse = cp.cp_lse_materialize(dm, ds)
+    lpkt, lpl = cp.cp_pack_from_lse(ov, lse, scatter_dim=scatter_dim)
+    r = 2
+    rpkt, rpl = cp.cp_pack_lse_rank(ov[r], dm[r], ds[r], W, scatter_dim=scatter_dim)
+    torch.cuda.synchronize()
+    ref_o, _, ref_l = orc.pack(o, m, s, scatter_dim)
+    assert np.array_equal(host_bits(pkt), ref_o), "packet payload differs"
+    check_pack_lse(pl.cpu().numpy(), ref_l, _packet_layout(m, W, T, H, scatter_dim),
+                   _packet_layout(s, W, T, H, scatter_dim))
+    assert torch.equal(lpkt.view(torch.int16), pkt.view(torch.int16))
+    assert torch.equal(rpkt.view(torch.int16), pkt[r].view(torch.int16))
+    assert torch.equal(rpl.view(torch.int32), pl[r].view(torch.int32))
+
+
 # ------------------------------------------------------------------------------------ permute
 
 @pytest.mark.parametrize("W,block_bytes", [(1, 48), (2, 16), (4, 4096), (5, 3), (8, 1000),
