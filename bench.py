@@ -1072,6 +1072,10 @@ def measure_breakdown(cp, wl, sets, stream, dev, peak):
         for ev in joined:
             stream.wait_event(ev)
     rec("pull_all_destinations", pull_all, wl.fused_bytes(), hold_ms=max(2.0, 0.1 * 20 * W))
+    res["pull_all_destinations"]["note"] = (
+        "one-GPU stand-in for the exchange across GPUs: W destination kernels on W streams, each "
+        "filling the GPU and reading one head chunk of every row from this GPU's HBM; across N "
+        "GPUs each destination reads (N-1)/N of its bytes over NVLink, which bounds it there")
     del pull_args, pstreams
     # context for the fused share at this size: a plain device-to-device copy
     # moving the fused kernel's byte count (half read, half written), timed the
