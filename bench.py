@@ -644,7 +644,7 @@ def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
     two must agree bit for bit on every rank."""
     import torch
     import torch.distributed as dist
-    from lse_pack_stable_b200.exchange import A2aExchange, PullExchange
+    from lse_pack_stable_b200.exchange import A2aExchange, PeerMapError, PullExchange
 
     wl = workload_for(args.config, world)
     if args.tokens > 0:
@@ -664,10 +664,20 @@ def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
     m_h = torch.from_numpy(mr).pin_memory()
     s_h = torch.from_numpy(sr).pin_memory()
 
-    pull = PullExchange(T, H, D, tdt, dev)
-    pull.o.view(torch.int16).copy_(o_h)
-    pull.smax.copy_(m_h)
-    pull.ssum.copy_(s_h)
+    # The pull path needs every rank's planes mapped into every process. If that
+    # fails on any rank, every rank learns it at the same point (PeerMapError)
+    # and the line times the NCCL path instead, saying why.
+    try:
+        pull, pull_error = PullExchange(T, H, D, tdt, dev), None
+        planes = (pull.o, pull.smax, pull.ssum)
+    except PeerMapError as e:
+        pull, pull_error = None, str(e)
+        planes = (torch.empty((T, H, D), dtype=tdt, device=dev),
+                  torch.empty((T, H), dtype=torch.float32, device=dev),
+                  torch.empty((T, H), dtype=torch.float32, device=dev))
+    planes[0].view(torch.int16).copy_(o_h)
+    planes[1].copy_(m_h)
+    planes[2].copy_(s_h)
     a2a = A2aExchange(T, H, D, tdt, dev)
     out_p = torch.empty((T, Hc, D), dtype=tdt, device=dev)
     lse_p = torch.empty((T, Hc), dtype=torch.float32, device=dev)
@@ -677,31 +687,43 @@ def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
     def barrier():
         dist.barrier()
 
+    def a2a_step(i):
+        a2a(*planes, out_a, lse_a)
+
+    if pull is not None:
+        def step(i):
+            pull(out_p, lse_p)
+    else:
+        step = a2a_step
+
     K, Wm = max(1, args.steps), max(3, args.warmup)
     # the two paths agree bit for bit (checked on every rank, then reduced)
-    pull(out_p, lse_p)
-    a2a(pull.o, pull.smax, pull.ssum, out_a, lse_a)
+    step(0)
+    a2a_step(0)
     torch.cuda.synchronize()
-    same = torch.tensor([float(torch.equal(out_p.view(torch.int16), out_a.view(torch.int16))
+    same = torch.tensor([float(pull is not None
+                               and torch.equal(out_p.view(torch.int16), out_a.view(torch.int16))
                                and torch.equal(lse_p.view(torch.int32), lse_a.view(torch.int32)))],
                         device=dev)
     dist.all_reduce(same, op=dist.ReduceOp.MIN)
 
     clocks = ClockSampler(dev.index)
     clocks.start()
-    pull_ms = time_back_to_back(lambda i: pull(out_p, lse_p), stream, K, Wm, barrier)
-    a2a_ms = time_back_to_back(lambda i: a2a(pull.o, pull.smax, pull.ssum, out_a, lse_a), stream,
-                               K, Wm, barrier)
+    pull_ms = time_back_to_back(step, stream, K, Wm, barrier)
+    a2a_ms = time_back_to_back(a2a_step, stream, K, Wm, barrier)
     # per call, the slowest rank (the FastVideo page's rank-max p50/p95)
-    pull_calls = rank_max_calls(lambda i: pull(out_p, lse_p), stream, K, world, dev)
-    a2a_calls = rank_max_calls(lambda i: a2a(pull.o, pull.smax, pull.ssum, out_a, lse_a), stream,
-                               K, world, dev)
+    pull_calls = rank_max_calls(step, stream, K, world, dev) if pull is not None else None
+    a2a_calls = rank_max_calls(a2a_step, stream, K, world, dev)
     clocks.stop()
     pull_ms, a2a_ms = reduce_max([pull_ms, a2a_ms], world, dev)
     bytes_per_call = wl.fused_bytes()                 # every rank's reads and writes together
     value = bytes_per_call * K / (pull_ms * 1e-3) / 1e9
-    # NVLink roofline: each destination reads (W-1) of its W contributions from peers
-    remote = (world - 1) * T * Hc * (2 * D + 8)
+    # NVLink roofline: each destination reads (W-1) of its W contributions from
+    # peers (pull); the all-to-all sends (W-1) of its W packet blocks
+    if pull is not None:
+        remote = (world - 1) * T * Hc * (2 * D + 8)
+    else:
+        remote = (world - 1) * T * Hc * (2 * D + 4)
     achieved = remote / (pull_ms / K * 1e-3) / 1e9
 
     # end to end through the public API: upload this rank's plane into its
@@ -710,12 +732,13 @@ def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
     hl = torch.empty((T, Hc), dtype=torch.float32, pin_memory=True)
 
     def e2e_step(i):
-        pull.o.view(torch.int16).copy_(o_h, non_blocking=True)
-        pull.smax.copy_(m_h, non_blocking=True)
-        pull.ssum.copy_(s_h, non_blocking=True)
-        pull(out_p, lse_p)
-        ho.copy_(out_p.view(torch.int16), non_blocking=True)
-        hl.copy_(lse_p, non_blocking=True)
+        planes[0].view(torch.int16).copy_(o_h, non_blocking=True)
+        planes[1].copy_(m_h, non_blocking=True)
+        planes[2].copy_(s_h, non_blocking=True)
+        step(i)
+        res_o, res_l = (out_p, lse_p) if pull is not None else (out_a, lse_a)
+        ho.copy_(res_o.view(torch.int16), non_blocking=True)
+        hl.copy_(res_l, non_blocking=True)
     ke = max(3, min(K, 20))
     e2e_ms = reduce_max([time_back_to_back(e2e_step, stream, ke, 3, barrier)], world, dev)[0]
     h2d = o_h.numel() * 2 + m_h.numel() * 4 + s_h.numel() * 4
@@ -731,15 +754,21 @@ def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
         "config": config_block(wl, world),
         "roofline": {"bound": "nvlink", "achieved": round(achieved, 2), "peak": NVLINK_PEER_GBS,
                      "unit": "GB/s", "frac": round(achieved / NVLINK_PEER_GBS, 4),
-                     "traffic": None, "kernel": "pull_combine_kernel (plain loads over NVLink)",
+                     "traffic": None,
+                     "kernel": ("pull_combine_kernel (plain loads over NVLink)" if pull is not None
+                                else "NCCL all-to-all between cp_pack_lse_rank and "
+                                     "cp_lse_combine_rank (pull path unavailable)"),
                      "peak_source": "measured B200 peer copy per direction (770 GB/s)",
                      "nvlink_bytes_per_rank_per_call": remote},
         "clocks": clocks.summary(), "gpu_launches": K,
         "e2e": {"value": round(bytes_per_call * ke / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world,
                 "ms_per_step": round(e2e_ms / ke, 4), "steps": ke},
-        "exchange": {"pull_equals_a2a": bool(same.item() == 1.0),
-                     "pull_rank_max_us_p50_p95": [round(1e3 * pct(pull_calls, q), 3) for q in (50, 95)],
+        "exchange": {"timed_path": "pull" if pull is not None else "a2a",
+                     "pull_unavailable": pull_error,
+                     "pull_equals_a2a": bool(same.item() == 1.0) if pull is not None else None,
+                     "pull_rank_max_us_p50_p95": ([round(1e3 * pct(pull_calls, q), 3) for q in (50, 95)]
+                                                  if pull_calls is not None else None),
                      "a2a_rank_max_us_p50_p95": [round(1e3 * pct(a2a_calls, q), 3) for q in (50, 95)],
                      "a2a_us_per_call": round(a2a_ms / K * 1e3, 3),
                      "a2a_GB/s": round(bytes_per_call * K / (a2a_ms * 1e-3) / 1e9, 2),
@@ -752,7 +781,8 @@ def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
     if rank == 0:
         print(json.dumps(line), flush=True)
     torch.cuda.synchronize()
-    pull.close()
+    if pull is not None:
+        pull.close()
     return 0
 
 
@@ -800,13 +830,16 @@ def measure_ulysses_exchange(wl, dev, stream, K, Wm, barrier, world):
     the NCCL all_to_all_4D; both must agree bit for bit."""
     import torch
     import torch.distributed as dist
-    from lse_pack_stable_b200.exchange import UlyssesPullExchange
+    from lse_pack_stable_b200.exchange import PeerMapError, UlyssesPullExchange
 
     rank = dist.get_rank()
     S, H, D = wl.T, wl.H, wl.D
     Bq, Bo = wl.ulysses_B
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float16
-    ex = UlyssesPullExchange(Bq, Bo, S, H, D, tdt, dev)
+    try:
+        ex = UlyssesPullExchange(Bq, Bo, S, H, D, tdt, dev)
+    except PeerMapError as e:       # raised on every rank alike
+        return {"unavailable": str(e)}
     wlr = synth.Workload(**{**wl.__dict__, "W": world})
     ex.seq.view(torch.int16).copy_(torch.from_numpy(
         synth.ulysses_seq_block(wlr, rank).view(np.int16)))

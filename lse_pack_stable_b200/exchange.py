@@ -143,39 +143,61 @@ def _stream_barrier(flag: torch.Tensor, group, stream=None) -> None:
         dist.all_reduce(flag, group=group)
 
 
+class PeerMapError(RuntimeError):
+    """Some rank of the group could not share or map the buffers; every rank
+    raises it at the same point, so that none is left waiting in a collective."""
+
+
 class PeerMap:
     """Tensors of this rank shared with every rank of the group: ``table(i)[r]``
     is rank r's tensor i -- this rank's own tensor, or the peer's mapped into
-    this process (a ``_Plane``). Construction and ``close`` are collective."""
+    this process (a ``_Plane``). Construction and ``close`` are collective.
+
+    The outcome is the group's, not this rank's: a failed export shows in the
+    gathered handles, a failed import in one all-reduce of a success flag, and
+    then every rank unmaps what it had mapped and raises ``PeerMapError``."""
 
     def __init__(self, tensors, group: Optional[dist.ProcessGroup] = None):
         self.group = group
         self.W = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         self.device = tensors[0].device
-        mine = [ipc_export(t) for t in tensors]
+        err: Optional[Exception] = None
+        try:
+            mine = [ipc_export(t) for t in tensors]
+        except CplseError as e:
+            mine, err = None, e
         every: List = [None] * self.W
         dist.all_gather_object(every, mine, group=group)
         self._bases: List[int] = []
         self._tables: List[List] = [[] for _ in tensors]
+        failed = [r for r in range(self.W) if every[r] is None]
+        if failed:
+            raise PeerMapError("rank(s) %s could not export their buffers%s"
+                               % (failed, ": %s" % err if err is not None else ""))
         for r in range(self.W):
             for i, t in enumerate(tensors):
                 if r == self.rank:
                     self._tables[i].append(t)
-                else:
-                    base, addr = ipc_import(every[r][i])
+                elif err is None:
+                    try:
+                        base, addr = ipc_import(every[r][i])
+                    except CplseError as e:
+                        err = e
+                        continue
                     self._bases.append(base)
                     self._tables[i].append(_Plane(addr, t))
+        ok = torch.tensor([0.0 if err is not None else 1.0], device=self.device)
+        dist.all_reduce(ok, op=dist.ReduceOp.MIN, group=group)
+        if ok.item() < 1.0:
+            self._unmap()
+            raise PeerMapError("mapping a peer's buffers failed on %s"
+                               % ("this rank: %s" % err if err is not None else "another rank"))
 
     def table(self, i: int) -> List:
         return self._tables[i]
 
-    def close(self) -> None:
-        """Unmap the peers' tensors, once every rank has finished reading."""
-        if not self._bases:
-            return
-        torch.cuda.synchronize(self.device)
-        dist.barrier(group=self.group)
+    def _unmap(self) -> None:
         err = None
         for b in self._bases:
             try:
@@ -185,6 +207,15 @@ class PeerMap:
         self._bases = []
         if err is not None:
             raise err
+
+    def close(self) -> None:
+        """Unmap the peers' tensors, once every rank has finished reading."""
+        if not self._bases:
+            return
+        if self.device.type == "cuda":
+            torch.cuda.synchronize(self.device)
+        dist.barrier(group=self.group)
+        self._unmap()
 
 
 class PullExchange:
