@@ -760,7 +760,9 @@ def run_exchange(args, cp, dev, rank, local_rank, world, peak, peak_kind):
                                      "cp_lse_combine_rank (pull path unavailable)"),
                      "peak_source": "measured B200 peer copy per direction (770 GB/s)",
                      "nvlink_bytes_per_rank_per_call": remote},
-        "clocks": clocks.summary(), "gpu_launches": K,
+        "clocks": clocks.summary(),
+        # this package's kernels per step: the pull kernel, or the per-rank pack and combine
+        "gpu_launches": K if pull is not None else 2 * K,
         "e2e": {"value": round(bytes_per_call * ke / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world,
                 "ms_per_step": round(e2e_ms / ke, 4), "steps": ke},
