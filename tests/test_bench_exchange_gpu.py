@@ -45,7 +45,7 @@ def test_bench_exchange_two_ranks_on_one_gpu(config, extra):
         assert rec["ulysses_exchange"]["pull_equals_nccl"] is True
 
 
-def _fallback_worker(rank, world, port, q):
+def _fallback_worker(rank, world, port, q, extra):
     import contextlib
     import io
     sys.path.insert(0, ROOT)
@@ -64,22 +64,25 @@ def _fallback_worker(rank, world, port, q):
         ex.ipc_import = import_refused_on_rank_1
         out = io.StringIO()
         with contextlib.redirect_stdout(out):
-            rc = bench.run_ours(bench.parse(["--gpus", "2", "--steps", "3", "--warmup", "3",
-                                             "--config", "decode"]))
+            rc = bench.run_ours(bench.parse(["--gpus", "2", "--steps", "3", "--warmup", "3"]
+                                            + extra))
         q.put((rank, rc, out.getvalue()))
     except Exception as e:  # noqa: BLE001
         q.put((rank, -1, repr(e)))
         raise
 
 
-def test_bench_exchange_falls_back_to_nccl_path_when_mapping_fails():
+@pytest.mark.parametrize("extra", [["--config", "decode"],
+                                   ["--config", "ulysses", "--tokens", "4096"]])
+def test_bench_exchange_falls_back_to_nccl_path_when_mapping_fails(extra):
     """One rank cannot map its peer's planes: every rank learns it at the same
-    point, no rank hangs, and the line times the all-to-all path and says why."""
+    point, no rank hangs, and the line times the all-to-all path and says why
+    (on Ulysses the load/store transforms say they were unavailable too)."""
     import torch.multiprocessing as mp
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_fallback_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_fallback_worker, args=(r, 2, port, q, extra)) for r in range(2)]
     for p in procs:
         p.start()
     got = {}
@@ -97,3 +100,5 @@ def test_bench_exchange_falls_back_to_nccl_path_when_mapping_fails():
     assert rec["exchange"]["pull_equals_a2a"] is None
     assert rec["value"] > 0 and "NCCL" in rec["roofline"]["kernel"]
     assert not [l for l in got[1][1].splitlines() if l.startswith("{")]   # rank 0 prints
+    if "ulysses" in extra:
+        assert "another rank" in rec["ulysses_exchange"]["unavailable"]
